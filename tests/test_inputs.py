@@ -1,0 +1,54 @@
+"""The seeded input generator (CPU only)."""
+import numpy as np
+
+from tree_speculative_decoding_05_b200 import inputs
+
+
+def test_splitmix64_reference_vector():
+    # splitmix64 from state 0: published first outputs of the generator.
+    got = [int(x) for x in inputs.raw_u64(np.uint64(0), 0, 3)]
+    assert got == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_bf16_rounding_is_rne():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 0.0, 65504.0])
+    got = inputs.to_bf16_bits(x)
+    assert list(got) == [0x3F80, 0x3F80, 0x3F82, 0xC020, 0x0000, 0x4780]
+    assert np.array_equal(inputs.bf16_bits_to_f64(got)[:4], [1.0, 1.0, 1.015625, -2.5])
+
+
+def test_normals_have_unit_moments():
+    z = inputs.normal(inputs.stream_base(3, 1), 200_000)
+    assert abs(z.mean()) < 0.01 and abs(z.std() - 1.0) < 0.01
+
+
+def test_random_trees_respect_limits():
+    for q in (9, 33, 65, 128):
+        p = inputs.random_parents(1, 0, q)
+        assert p[0] == -1 and all(0 <= p[i] < i for i in range(1, q))
+        depth = np.zeros(q, int)
+        for i in range(1, q):
+            depth[i] = depth[p[i]] + 1
+        assert depth.max() <= inputs.MAX_DEPTH
+
+
+def test_planted_chain_and_tokens():
+    w = inputs.config(4, prefix_lens=[64])
+    chain = w.forced_path[0]
+    assert len(chain) == 16 and chain[0] == 0 and (np.diff(chain) > 0).all()
+    for a, c in zip(chain[:-1], chain[1:]):
+        assert w.parents[0, c] == a and w.target_tokens[0, a] == w.node_tokens[0, c]
+
+
+def test_retrieve_pointers_enumerate_children_in_order():
+    p = np.array([-1, 0, 0, 1, 0, 3], np.int32)
+    first, sib = inputs.retrieve_pointers(p)
+    assert list(first) == [1, 3, -1, 5, -1, -1]
+    assert list(sib) == [-1, 2, 4, -1, -1, -1]
+
+
+def test_workload_is_deterministic():
+    a = inputs.config(0)
+    b = inputs.config(0)
+    assert np.array_equal(a.q_lat, b.q_lat) and np.array_equal(a.c_kv, b.c_kv)
+    assert a.c_kv.shape == (1, 265, 512) and a.q_lat.shape == (1, 9, 64, 512)

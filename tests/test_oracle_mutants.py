@@ -1,0 +1,45 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch
+every one of them (CPU only; the planted copy lives in a temporary directory)."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ddt_oracle.c")
+
+# (name, text to replace, replacement).  Each is a mistake a port could make.
+MUTANTS = [
+    ("drop rope term", "dot += bf16_to_double(qr[d]) * bf16_to_double(rrow[d]);", ";"),
+    ("drop softmax scale", "s[j] = scale * dot;", "s[j] = dot;"),
+    ("node does not see itself", "vis[(size_t)i * Q + i] = 1;", ";"),
+    ("tree rows reversed", "vis_row[j - P]", "vis_row[T - 1 - j]"),
+    ("lse without the max", "*lse = m + log(Z);", "*lse = log(Z);"),
+    ("value from the wrong row", "const uint16_t* vrow = ckv + (int64_t)j * ckv_rs;",
+     "const uint16_t* vrow = ckv + (int64_t)(j > 0 ? j - 1 : 0) * ckv_rs;"),
+    ("mask bit order", "word |= (uint64_t)1 << k;", "word |= (uint64_t)1 << (63 - k);"),
+    ("accept compares with the wrong target", "if (tok[c] == tgt[cur])", "if (tok[c] == tgt[c])"),
+    ("accept skips the first child", "int c = first[cur];", "int c = first[cur] == -1 ? -1 : sib[first[cur]];"),
+    ("compaction writes one row late", "memcpy(ckv + (int64_t)(P + i) * ckv_rs",
+     "memcpy(ckv + (int64_t)(P + i + (i + 1 < alen)) * ckv_rs"),
+    ("depth off by one", "depth[i] = (i == 0) ? 0 : depth[parents[i]] + 1;",
+     "depth[i] = (i == 0) ? 1 : depth[parents[i]] + 1;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.compile_oracle(str(path), str(tmp_path / "libmutant.so"))
+    orc = oracle.Oracle(lib)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake '{name}'"
