@@ -1,0 +1,502 @@
+"""Benchmark of the tree-verify step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ddt,reference}]
+                    [--config 2] [--no-cpu-baseline] [--no-e2e]
+
+One step is one pass of the whole verification path over one synthetic batch:
+visibility mask -> tree-verify attention (with its split merge when used) ->
+greedy accept -> KV compaction.  The default workload is 64 requests x q_len 33
+(64 heads) x prefix 4096.  Prints one JSON line (rank 0).
+
+value        verify-attention algorithmic TFLOP/s of the whole job: FLOPs of all
+             ranks' steps / the max over ranks of the device-timed step time.
+ms_per_step  device time of one step (CUDA events, max over ranks).
+roofline     the verify kernel alone: algorithmic FLOPs per launch / its mean
+             launch time (CUDA events on its stream) against the measured bf16
+             dense peak.
+e2e          the same metric through the public API with host buffers: each step
+             copies its per-step inputs from pinned host memory, runs the step
+             and reads the accepted tokens back.
+cpu_baseline the CPU oracle on a bounded sample of the same workload (rank 0).
+
+With N > 1 (torchrun) every rank runs its own batch (replicas, weak scaling);
+there is no collective on the data path, only the timing reduction.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "verify-attn µs/call & TFLOP/s (% bf16 peak), 64 streams × q_len 33 × 4K prefix"
+H, DL, DR = 64, 512, 64
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ---------------------------------------------------------------------------
+# Work accounting (host side, from the workload's tree shapes)
+# ---------------------------------------------------------------------------
+
+def tree_depths(parents: np.ndarray) -> np.ndarray:
+    depth = np.zeros_like(parents)
+    for b in range(parents.shape[0]):
+        for i in range(1, parents.shape[1]):
+            depth[b, i] = depth[b, parents[b, i]] + 1
+    return depth
+
+
+def verify_flops(prefix_lens: np.ndarray, parents: np.ndarray, heads: int = H) -> float:
+    """Algorithmic FLOPs of one verify call: every (request, node, head) row does a
+    576-wide dot product and a 512-wide accumulation per visible key; masked keys
+    are not counted.  Visible keys of node i: P + depth(i) + 1."""
+    depth = tree_depths(parents)
+    visible = prefix_lens[:, None].astype(np.float64) + depth + 1
+    return float(heads * 2 * (DL + DR + DL) * visible.sum())
+
+
+def verify_bytes(prefix_lens: np.ndarray, q_len: int, out_bytes: int, want_lse: bool) -> float:
+    """Algorithmic bytes: queries read once, each request's KV rows read once,
+    outputs (and lse) written once."""
+    B = prefix_lens.shape[0]
+    q = B * q_len * H * (DL + DR) * 2
+    kv = float((prefix_lens.astype(np.float64) + q_len).sum()) * (DL + DR) * 2
+    out = B * q_len * H * DL * out_bytes + (B * q_len * H * 4 if want_lse else 0)
+    return q + kv + out
+
+
+def flops_rows(prefix_lens, parents, rows, heads=H) -> float:
+    """FLOPs of a subset of query rows (flat (b*Q + i)*H + h)."""
+    depth = tree_depths(parents)
+    Q = parents.shape[1]
+    b = rows // (Q * heads)
+    i = (rows // heads) % Q
+    vis = prefix_lens[b].astype(np.float64) + depth[b, i] + 1
+    return float(2 * (DL + DR + DL) * vis.sum())
+
+
+# ---------------------------------------------------------------------------
+# Peaks and clocks
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def physical_gpu_index(local: int) -> str:
+    """nvidia-smi's index of the GPU this process uses."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (timing reduction only)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(values: list[float], world: int, device) -> list[float]:
+    """Element-wise max over ranks (identity on one rank)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def reduce_sum(values: list[float], world: int, device) -> list[float]:
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.cpu()]
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+def oracle_sample_throughput(w, target_seconds: float, seed: int = 0, max_rows: int = 1 << 16):
+    """Run the CPU oracle on random query rows of the workload until about
+    target_seconds of CPU work; returns (TFLOP/s, rows, seconds, threads)."""
+    import oracle
+    rng = np.random.RandomState(seed)
+    total = w.B * w.q_len * H
+    done_rows, flops, secs = 0, 0.0, 0.0
+    chunk = max(16, oracle.threads() * 4)
+    while secs < target_seconds and done_rows < max_rows:
+        rows = np.sort(rng.choice(total, size=min(chunk, total), replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens, w.parents,
+                         w.softmax_scale, rows)
+        secs += time.perf_counter() - t0
+        flops += flops_rows(w.prefix_lens, w.parents, rows)
+        done_rows += len(rows)
+        chunk = min(chunk * 2, 4096)
+    return flops / secs / 1e12, done_rows, secs, oracle.threads()
+
+
+def run_reference(args, w):
+    """--impl reference: the CPU oracle as it stands, each step a bounded sample
+    (query rows of the attention, plus the mask/accept/compaction of the batch)."""
+    import oracle
+    rows_per_step = max(32, oracle.threads() * 8)
+    total = w.B * w.q_len * H
+    rng = np.random.RandomState(1)
+
+    def step():
+        rows = np.sort(rng.choice(total, size=rows_per_step, replace=False)).astype(np.int64)
+        oracle.build_mask(w.parents)
+        oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens, w.parents,
+                         w.softmax_scale, rows)
+        path, alen, _, _ = oracle.tree_accept(w.node_tokens, w.target_tokens, w.next_token,
+                                              w.next_sibling)
+        oracle.kv_compact(w.c_kv, w.k_rope, w.prefix_lens, path, alen)
+        return flops_rows(w.prefix_lens, w.parents, rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += step()
+    secs = time.perf_counter() - t0
+    value = flops / secs / 1e12
+    sample = (f"{rows_per_step} random query rows of the attention per step "
+              f"(of {total}) + mask, accept and compaction of the full batch")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "q_len": w.q_len, "heads": H,
+                   "prefix": int(w.prefix_lens.max()), "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Main (GPU arm)
+# ---------------------------------------------------------------------------
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ddt", "reference"], default="ddt")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_env()
+    from tree_speculative_decoding_05_b200 import inputs
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        run_reference(args, inputs.config(args.config))
+        return 0
+
+    import torch
+
+    from tree_speculative_decoding_05_b200 import ddt
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    # Every rank runs its own batch of the same shape (independent requests).
+    w = inputs.config(args.config)
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32))
+
+    host = {
+        "q_lat": bf16(w.q_lat), "q_rope": bf16(w.q_rope), "c_kv": bf16(w.c_kv),
+        "k_rope": bf16(w.k_rope), "prefix": i32(w.prefix_lens), "parents": i32(w.parents),
+        "node_tokens": i32(w.node_tokens), "target_tokens": i32(w.target_tokens),
+        "next_token": i32(w.next_token), "next_sibling": i32(w.next_sibling),
+    }
+    d = {k: v.to(device) for k, v in host.items()}
+    out_dtype = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    B, Q = w.B, w.q_len
+    max_prefix = int(w.prefix_lens.max())
+    mask = torch.empty((B, Q, (Q + 63) // 64), dtype=torch.int64, device=device)
+    depth = torch.empty((B, Q), dtype=torch.int32, device=device)
+    mstatus = torch.empty((B,), dtype=torch.int32, device=device)
+    out = torch.empty((B, Q, H, DL), dtype=out_dtype, device=device)
+    lse = torch.empty((B, Q, H), dtype=torch.float32, device=device) if w.want_lse else None
+    vstatus = torch.empty((B,), dtype=torch.int32, device=device)
+    ws_bytes, splits = ddt.verify_attn_workspace_size(
+        d["q_lat"], d["q_rope"], d["c_kv"], d["k_rope"], d["prefix"], mask, w.softmax_scale,
+        max_prefix)
+    workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    path = torch.empty((B, Q), dtype=torch.int32, device=device)
+    alen = torch.empty((B,), dtype=torch.int32, device=device)
+    bonus = torch.empty((B,), dtype=torch.int32, device=device)
+    astatus = torch.empty((B,), dtype=torch.int32, device=device)
+    newp = torch.empty((B,), dtype=torch.int32, device=device)
+    cstatus = torch.empty((B,), dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        ddt.build_mask(d["parents"], mask=mask, depth=depth, status=mstatus)
+        if ev is not None:
+            ev[0].record(stream)
+        ddt.verify_attn(d["q_lat"], d["q_rope"], d["c_kv"], d["k_rope"], d["prefix"], mask,
+                        w.softmax_scale, max_prefix=max_prefix, out=out, lse=lse,
+                        workspace=workspace if ws_bytes else None, status=vstatus)
+        if ev is not None:
+            ev[1].record(stream)
+        ddt.tree_accept(d["node_tokens"], d["target_tokens"], d["next_token"],
+                        d["next_sibling"], path=path, accept_len=alen, bonus=bonus,
+                        status=astatus)
+        ddt.kv_compact(d["c_kv"], d["k_rope"], d["prefix"], path, alen, new_prefix_lens=newp,
+                       status=cstatus)
+
+    launches_per_step = 4 + (1 if splits > 1 else 0)
+    ddt.fault_flags(reset=True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(physical_gpu_index(local)) as clocks:
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    verify_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    faults = ddt.fault_flags(reset=True)
+    statuses_ok = all(int(s.max()) == 0 for s in (mstatus, vstatus, astatus, cstatus))
+
+    flops_local = verify_flops(w.prefix_lens, w.parents)
+    bytes_local = verify_bytes(w.prefix_lens, Q, 4 if out_dtype == torch.float32 else 2,
+                               w.want_lse)
+    step_ms_max, verify_ms_max = reduce_max([step_ms, verify_ms], world, device)
+    flops_total = reduce_sum([flops_local], world, device)[0]
+
+    # ---- end to end through the public API with host buffers ---------------
+    e2e = None
+    if not args.no_e2e:
+        tree_rows = np.stack([np.arange(int(p), int(p) + Q) for p in w.prefix_lens])
+        pin = {k: host[k].pin_memory() for k in ("q_lat", "q_rope", "parents", "node_tokens",
+                                                 "target_tokens", "next_token", "next_sibling",
+                                                 "prefix")}
+        tree_ckv = host["c_kv"][torch.arange(B)[:, None], torch.from_numpy(tree_rows)].pin_memory()
+        tree_kr = host["k_rope"][torch.arange(B)[:, None], torch.from_numpy(tree_rows)].pin_memory()
+        idx = torch.from_numpy(tree_rows).to(device)
+        bidx = torch.arange(B, device=device)[:, None]
+        res_host = {k: torch.empty_like(v, device="cpu").pin_memory()
+                    for k, v in (("path", path), ("alen", alen), ("bonus", bonus), ("newp", newp))}
+        d2h = sum(v.numel() * v.element_size() for v in res_host.values())
+        h2d = sum(v.numel() * v.element_size() for v in pin.values()) + \
+            tree_ckv.numel() * 2 + tree_kr.numel() * 2
+        dev_tree_ckv = torch.empty_like(tree_ckv, device=device)
+        dev_tree_kr = torch.empty_like(tree_kr, device=device)
+
+        def e2e_step():
+            for k, v in pin.items():
+                d[k].copy_(v, non_blocking=True)
+            dev_tree_ckv.copy_(tree_ckv, non_blocking=True)
+            dev_tree_kr.copy_(tree_kr, non_blocking=True)
+            d["c_kv"][bidx, idx] = dev_tree_ckv
+            d["k_rope"][bidx, idx] = dev_tree_kr
+            step()
+            for k, src in (("path", path), ("alen", alen), ("bonus", bonus), ("newp", newp)):
+                res_host[k].copy_(src, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max([e0.elapsed_time(e1) / args.steps], world, device)[0]
+        e2e = {"value": flops_total / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms,
+               "resident": "prefix KV rows stay in HBM (the cache); per step the queries, "
+                           "the tree block's KV rows and the tree arrays are copied in and "
+                           "the accepted tokens read back"}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, rows, secs, cores = oracle_sample_throughput(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} random query rows of the workload's attention "
+                         f"({secs:.1f} s, fp64 C oracle, OpenMP)"}
+
+    if rank == 0:
+        peaks, peak_src = measured_peaks()
+        timed_s = step_ms * args.steps / 1e3
+        use_sustained = timed_s > 2.0
+        peak = peaks.get("bf16_tflops_sustained" if use_sustained else "bf16_tflops",
+                         FALLBACK_BF16_TFLOPS)
+        achieved = flops_local / (verify_ms_max * 1e-3) / 1e12
+        clk = clocks.summary()
+        line = {
+            "metric": METRIC,
+            "value": flops_total / (step_ms_max * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": step_ms_max,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "q_len": Q, "heads": H,
+                       "prefix": max_prefix, "out": w.out_dtype, "kv_splits": splits,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (KV %.0f MB + queries %.0f MB per GPU); "
+                             "no flush" % (w.c_kv.nbytes / 1e6 + w.k_rope.nbytes / 1e6,
+                                           (w.q_lat.nbytes + w.q_rope.nbytes) / 1e6)},
+            "verify_us_per_call": verify_ms_max * 1e3,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peak_src} {'sustained' if use_sustained else 'burst'} bf16",
+                         "traffic": None,
+                         "algorithmic_bytes": bytes_local,
+                         "kernel": "verify_attn_kernel"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
+                       "reasons": clk["reasons"]},
+            "faults": faults,
+            "statuses_ok": statuses_ok,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

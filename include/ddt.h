@@ -46,6 +46,13 @@
 extern "C" {
 #endif
 
+/* Symbols of the shared library. */
+#if defined(__GNUC__)
+#define DDT_API __attribute__((visibility("default")))
+#else
+#define DDT_API
+#endif
+
 /* Opaque CUDA stream: identical to cudaStream_t / CUstream. */
 struct CUstream_st;
 typedef struct CUstream_st* ddt_stream_t;
@@ -98,7 +105,7 @@ typedef enum ddt_dtype { DDT_F32 = 0, DDT_BF16 = 1 } ddt_dtype;
  *          that request's mask words are all 0 and its depths are all -1.
  * Errors: B < 0, q_len outside [1,128], parents or mask NULL with B > 0 ->
  *         DDT_ERR_INVALID_ARG / DDT_ERR_UNSUPPORTED.  B = 0 is a no-op. */
-ddt_status ddt_build_mask(const int32_t* parents, int32_t B, int32_t q_len,
+DDT_API ddt_status ddt_build_mask(const int32_t* parents, int32_t B, int32_t q_len,
                           uint64_t* mask, int32_t* depth, int32_t* status,
                           ddt_stream_t stream);
 
@@ -162,12 +169,12 @@ typedef struct ddt_attn_args {
 } ddt_attn_args;
 
 /* Bytes of workspace the call will use for these arguments (0 if no split). */
-size_t ddt_verify_attn_workspace_size(const ddt_attn_args* args);
+DDT_API size_t ddt_verify_attn_workspace_size(const ddt_attn_args* args);
 
 /* Number of KV splits the call will use for these arguments. */
-int32_t ddt_verify_attn_num_splits(const ddt_attn_args* args);
+DDT_API int32_t ddt_verify_attn_num_splits(const ddt_attn_args* args);
 
-ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t stream);
+DDT_API ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* ddt_tree_accept                                                          */
@@ -196,7 +203,7 @@ ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t stream);
  * node_tokens, target_tokens, next_token, next_sibling: int32 [B, q_len].
  * path int32 [B, q_len]; accept_len, bonus_token, status: int32 [B]
  * (bonus_token and status may be NULL). */
-ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* target_tokens,
+DDT_API ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* target_tokens,
                            const int32_t* next_token, const int32_t* next_sibling,
                            int32_t B, int32_t q_len, int32_t* path, int32_t* accept_len,
                            int32_t* bonus_token, int32_t* status, ddt_stream_t stream);
@@ -225,7 +232,7 @@ ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* target_tok
  * outside [0, q_len)) or DDT_REQ_BAD_PREFIX (P < 0 or P + q_len > capacity);
  * a request with a non-zero status is left unchanged and its new prefix equals
  * its old one. */
-ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
+DDT_API ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
                           int64_t ckv_row_stride, int64_t kr_batch_stride,
                           int64_t kr_row_stride, int32_t capacity,
                           const int32_t* prefix_lens, const int32_t* path,
@@ -234,10 +241,17 @@ ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
                           ddt_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
-const char* ddt_status_str(ddt_status status);
+DDT_API const char* ddt_status_str(ddt_status status);
+
+/* Diagnostic: the library's device fault word, a bit set of
+ *   1 = a kernel gave up waiting on a barrier (bounded wait expired).
+ * Reading it synchronises the device; with reset != 0 it is cleared.  A clean
+ * run leaves it 0. */
+#define DDT_FAULT_WAIT_TIMEOUT 1u
+DDT_API ddt_status ddt_fault_flags(uint32_t* flags, int32_t reset);
 
 /* Library version string (static storage). */
-const char* ddt_version(void);
+DDT_API const char* ddt_version(void);
 
 #ifdef __cplusplus
 }

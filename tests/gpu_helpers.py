@@ -1,0 +1,81 @@
+"""Helpers of the GPU parity tests: move a seeded workload to the device, run the
+library's calls, and compare with the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from tree_speculative_decoding_05_b200 import ddt, inputs
+
+# Tolerances for the attention output against the float64 oracle (bf16 P and,
+# for bf16 outputs, the final rounding dominate; see the design doc readings).
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+LSE_MAX_ABS = 5e-3
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).to(device)
+
+
+def i32(a, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+
+class DeviceWorkload:
+    def __init__(self, w: inputs.Workload, device="cuda"):
+        self.w = w
+        self.q_lat = bf16_tensor(w.q_lat, device)
+        self.q_rope = bf16_tensor(w.q_rope, device)
+        self.c_kv = bf16_tensor(w.c_kv, device)
+        self.k_rope = bf16_tensor(w.k_rope, device)
+        self.prefix = i32(w.prefix_lens, device)
+        self.parents = i32(w.parents, device)
+        self.node_tokens = i32(w.node_tokens, device)
+        self.target_tokens = i32(w.target_tokens, device)
+        self.next_token = i32(w.next_token, device)
+        self.next_sibling = i32(w.next_sibling, device)
+
+    def verify(self, num_splits=0, out_dtype=None, want_lse=None, mask=None):
+        w = self.w
+        if mask is None:
+            mask, _, _ = ddt.build_mask(self.parents)
+        od = out_dtype or (torch.float32 if w.out_dtype == "f32" else torch.bfloat16)
+        status = torch.empty(w.B, dtype=torch.int32, device=self.q_lat.device)
+        out, lse = ddt.verify_attn(self.q_lat, self.q_rope, self.c_kv, self.k_rope, self.prefix,
+                                   mask, w.softmax_scale, max_prefix=int(w.prefix_lens.max()),
+                                   out_dtype=od, want_lse=True if want_lse is None else want_lse,
+                                   num_splits=num_splits, status=status)
+        return out, lse, status
+
+
+def compare_attention(out_gpu: np.ndarray, ref: np.ndarray, what: str = ""):
+    """Max-abs and relative-L2 error of a GPU result against float64 values."""
+    g = out_gpu.astype(np.float64)
+    err = np.abs(g - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(g - ref) / denom) if denom > 0 else float(np.linalg.norm(g - ref))
+    assert np.isfinite(g).all(), f"{what}: non-finite output"
+    assert max_abs <= MAX_ABS, f"{what}: max abs err {max_abs:.3e} > {MAX_ABS}"
+    assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e} > {REL_L2}"
+    return max_abs, rel
+
+
+def rows_of(out: torch.Tensor, rows: np.ndarray) -> np.ndarray:
+    flat = out.reshape(-1, out.shape[-1])
+    idx = torch.from_numpy(rows).to(out.device)
+    return flat.index_select(0, idx).float().cpu().numpy()
+
+
+def sample_rows(B, Q, H, n, seed=0, must=()):
+    """n distinct flat rows (b*Q + i)*H + h, always including `must`."""
+    total = B * Q * H
+    rng = np.random.RandomState(seed)
+    pick = set(int(r) for r in must if 0 <= r < total)
+    if n >= total:
+        return np.arange(total, dtype=np.int64)
+    while len(pick) < n:
+        pick.add(int(rng.randint(total)))
+    return np.array(sorted(pick), dtype=np.int64)

@@ -1,0 +1,69 @@
+"""The multi-GPU path on the CPU: requests are independent, so N GPUs run N
+replicas and the only cross-rank step is the timing reduction (max of the step
+times, sum of the work).  Checked here with world_size 2 over gloo."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+
+    w, r, _ = bench.dist_env()
+    dist = bench.init_dist(w, "gloo")
+    try:
+        step_ms = [2.0, 3.5][rank]
+        verify_ms = [1.5, 1.0][rank]
+        mx = bench.reduce_max([step_ms, verify_ms], w, "cpu")
+        sm = bench.reduce_sum([10.0 * (rank + 1)], w, "cpu")
+        q.put((r, mx, sm))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_timing_reduction_over_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, mx, sm in results:
+        assert mx == [3.5, 1.5]          # each quantity's max over ranks
+        assert sm == [30.0]
+
+
+def test_single_rank_reduction_is_identity():
+    import bench
+    assert bench.reduce_max([1.0, 2.0], 1, "cpu") == [1.0, 2.0]
+    assert bench.reduce_sum([4.0], 1, "cpu") == [4.0]
+
+
+def test_work_accounting_matches_definition():
+    """FLOPs per verify call: 64 heads x 2 x (576 + 512) per visible key, where
+    node i sees P + depth(i) + 1 keys (chain tree: depth(i) = i)."""
+    import numpy as np
+
+    import bench
+    from tree_speculative_decoding_05_b200 import inputs
+    parents = np.stack([inputs.chain_parents(5), inputs.star_parents(5)])
+    prefix = np.array([10, 0], np.int32)
+    f = bench.verify_flops(prefix, parents)
+    vis = (10 * 5 + sum(range(1, 6))) + (1 + 2 * 4)
+    assert f == 64 * 2 * 1088 * vis
+    rows = np.arange(2 * 5 * 64)
+    assert bench.flops_rows(prefix, parents, rows) == pytest.approx(f)

@@ -1,0 +1,183 @@
+// api.cu — the extern "C" entry points of libddt: host-side argument checks,
+// then one launch per call on the caller's stream.  No entry point allocates
+// device memory or synchronises the host.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "ddt.h"
+#include "ddt_internal.h"
+
+namespace ddt {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSlots = 8;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared cache row checks of ddt_verify_attn and ddt_kv_compact.
+bool cache_strides_ok(int B, int capacity, int64_t ckv_bs, int64_t ckv_rs, int64_t kr_bs,
+                      int64_t kr_rs) {
+  if (ckv_rs < DDT_D_LATENT || kr_rs < DDT_D_ROPE) return false;
+  if ((ckv_rs % 8) || (kr_rs % 8) || (ckv_bs % 8) || (kr_bs % 8)) return false;
+  if (B > 1 && (ckv_bs < static_cast<int64_t>(capacity) * ckv_rs ||
+                kr_bs < static_cast<int64_t>(capacity) * kr_rs))
+    return false;
+  return true;
+}
+
+}  // namespace
+
+int device_sm_count() {
+  static int counts[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+cudaError_t ensure_smem_limit(const void* func, int bytes, int slot) {
+  static std::mutex mu;
+  static bool done[kMaxDevices][kMaxSlots] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices || slot < 0 || slot >= kMaxSlots)
+    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev][slot]) {
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev][slot] = true;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace ddt
+
+using namespace ddt;
+
+extern "C" {
+
+const char* ddt_version(void) { return "ddt 0.1.0 (sm_100a)"; }
+
+const char* ddt_status_str(ddt_status s) {
+  switch (s) {
+    case DDT_OK: return "ok";
+    case DDT_ERR_INVALID_ARG: return "invalid argument";
+    case DDT_ERR_UNSUPPORTED: return "unsupported shape";
+    case DDT_ERR_CUDA: return "CUDA error";
+    case DDT_ERR_INPUT: return "malformed request data";
+  }
+  return "unknown status";
+}
+
+ddt_status ddt_build_mask(const int32_t* parents, int32_t B, int32_t q_len, uint64_t* mask,
+                          int32_t* depth, int32_t* status, ddt_stream_t stream) {
+  if (B < 0) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!parents || !mask) return DDT_ERR_INVALID_ARG;
+  if (launch_build_mask(parents, B, q_len, mask, depth, status,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
+ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* target_tokens,
+                           const int32_t* next_token, const int32_t* next_sibling, int32_t B,
+                           int32_t q_len, int32_t* path, int32_t* accept_len,
+                           int32_t* bonus_token, int32_t* status, ddt_stream_t stream) {
+  if (B < 0) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!node_tokens || !target_tokens || !next_token || !next_sibling || !path || !accept_len)
+    return DDT_ERR_INVALID_ARG;
+  if (launch_tree_accept(node_tokens, target_tokens, next_token, next_sibling, B, q_len, path,
+                         accept_len, bonus_token, status,
+                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
+ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
+                          int64_t ckv_row_stride, int64_t kr_batch_stride, int64_t kr_row_stride,
+                          int32_t capacity, const int32_t* prefix_lens, const int32_t* path,
+                          const int32_t* accept_len, int32_t B, int32_t q_len,
+                          int32_t* new_prefix_lens, int32_t* status, ddt_stream_t stream) {
+  if (B < 0 || capacity < 0) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!c_kv || !k_rope || !prefix_lens || !path || !accept_len) return DDT_ERR_INVALID_ARG;
+  if (!aligned16(c_kv) || !aligned16(k_rope)) return DDT_ERR_INVALID_ARG;
+  if (!cache_strides_ok(B, capacity, ckv_batch_stride, ckv_row_stride, kr_batch_stride,
+                        kr_row_stride))
+    return DDT_ERR_INVALID_ARG;
+  if (launch_kv_compact(static_cast<uint16_t*>(c_kv), static_cast<uint16_t*>(k_rope),
+                        ckv_batch_stride, ckv_row_stride, kr_batch_stride, kr_row_stride, capacity,
+                        prefix_lens, path, accept_len, B, q_len, new_prefix_lens, status,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
+static ddt_status check_attn_args(const ddt_attn_args* a) {
+  if (!a) return DDT_ERR_INVALID_ARG;
+  if (a->B < 0 || a->capacity < 0 || a->max_prefix < 0) return DDT_ERR_INVALID_ARG;
+  if (a->q_len < 1 || a->q_len > DDT_MAX_Q_LEN || a->num_heads != DDT_NUM_HEADS ||
+      a->d_latent != DDT_D_LATENT || a->d_rope != DDT_D_ROPE)
+    return DDT_ERR_UNSUPPORTED;
+  if (a->out_dtype != DDT_F32 && a->out_dtype != DDT_BF16) return DDT_ERR_INVALID_ARG;
+  if (a->num_splits < 0 || a->num_splits > 64) return DDT_ERR_INVALID_ARG;
+  if (a->B == 0) return DDT_OK;
+  if (!a->prefix_lens || !a->q_lat || !a->q_rope || !a->c_kv || !a->k_rope || !a->mask || !a->out)
+    return DDT_ERR_INVALID_ARG;
+  if (!aligned16(a->q_lat) || !aligned16(a->q_rope) || !aligned16(a->c_kv) ||
+      !aligned16(a->k_rope) || !aligned16(a->out))
+    return DDT_ERR_INVALID_ARG;
+  if (a->capacity < a->q_len) return DDT_ERR_INVALID_ARG;
+  if (!cache_strides_ok(a->B, a->capacity, a->ckv_batch_stride, a->ckv_row_stride,
+                        a->kr_batch_stride, a->kr_row_stride))
+    return DDT_ERR_INVALID_ARG;
+  if (!(a->softmax_scale == a->softmax_scale)) return DDT_ERR_INVALID_ARG;
+  return DDT_OK;
+}
+
+int32_t ddt_verify_attn_num_splits(const ddt_attn_args* a) {
+  if (check_attn_args(a) != DDT_OK || a->B == 0) return 1;
+  return verify_num_splits(*a, device_sm_count());
+}
+
+size_t ddt_verify_attn_workspace_size(const ddt_attn_args* a) {
+  if (check_attn_args(a) != DDT_OK || a->B == 0) return 0;
+  return verify_workspace_bytes(*a, verify_num_splits(*a, device_sm_count()));
+}
+
+ddt_status ddt_verify_attn(const ddt_attn_args* a, ddt_stream_t stream) {
+  const ddt_status st = check_attn_args(a);
+  if (st != DDT_OK || a->B == 0) return st;
+  int splits = verify_num_splits(*a, device_sm_count());
+  const size_t need = verify_workspace_bytes(*a, splits);
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  if (splits > 1) {
+    if (!a->workspace || a->workspace_bytes < need ||
+        (reinterpret_cast<uintptr_t>(a->workspace) & 255u)) {
+      splits = 1;
+    } else {
+      part_o = static_cast<float*>(a->workspace);
+      part_lse = part_o + static_cast<size_t>(splits) * a->B * a->q_len * 64 * 512;
+    }
+  }
+  return launch_verify_attn(*a, splits, part_o, part_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,246 @@
+// companions.cu — the integer kernels of the tree-verify step: visibility mask,
+// greedy tree accept, and KV-cache compaction.  All three are bit-exact by
+// construction (pure integer / bit-copy work) and bounded on any input.
+//
+// Sources (page title, section):
+//   [Race Conditions] "Race Conditions, Buffer Aliasing, and the Architecture of
+//       a Native DDTree Inference Engine"
+//   [Foundation] "Building the Foundation: Architecting a Native CUDA DDTree
+//       Inference Engine"
+//   [Verdict] "The Microsecond Verdict: Validating a DDTree Kernel Fix Under
+//       Time Pressure"
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ddt.h"
+#include "ddt_internal.h"
+
+namespace ddt {
+
+// ---------------------------------------------------------------------------
+// Visibility mask.  [Foundation] "The Single-Threaded Heap Design": the block's
+// threads build the visibility matrix in parallel; [Race Conditions] "The
+// Cache Compaction Problem": parents precede children.  One CTA per request,
+// thread i builds row i by walking i's parent chain (at most i steps once the
+// parents are validated, since parents[k] < k).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) build_mask_kernel(const int32_t* __restrict__ parents,
+                                                         int q_len, uint64_t* __restrict__ mask,
+                                                         int32_t* __restrict__ depth,
+                                                         int32_t* __restrict__ status) {
+  __shared__ int32_t s_par[DDT_MAX_Q_LEN];
+  const int b = blockIdx.x;
+  const int i = threadIdx.x;
+  const int W = (q_len + 63) >> 6;
+  int ok = 1;
+  if (i < q_len) {
+    const int32_t p = parents[static_cast<int64_t>(b) * q_len + i];
+    s_par[i] = p;
+    ok = (i == 0) ? (p == -1) : (p >= 0 && p < i);
+  }
+  const int all_ok = __syncthreads_and(ok);
+  if (i >= q_len) return;
+  uint64_t w0 = 0, w1 = 0;
+  int d = -1;
+  if (all_ok) {
+    int a = i;
+    d = 0;
+    for (int step = 0; step <= i; ++step) {  // bounded: the chain strictly decreases
+      if (a < 64) w0 |= 1ull << a;
+      else w1 |= 1ull << (a - 64);
+      if (a == 0) break;
+      a = s_par[a];
+      ++d;
+    }
+  }
+  uint64_t* row = mask + (static_cast<int64_t>(b) * q_len + i) * W;
+  row[0] = w0;
+  if (W > 1) row[1] = w1;
+  if (depth) depth[static_cast<int64_t>(b) * q_len + i] = d;
+  if (status && i == 0) status[b] = all_ok ? DDT_REQ_OK : DDT_REQ_BAD_PARENT;
+}
+
+// ---------------------------------------------------------------------------
+// Greedy accept.  [Verdict] "The Crash That Demanded a Fix" and "What Was
+// Learned": follow the first-child / next-sibling retrieve pointers, accept the
+// child whose draft token equals the target's greedy token, stop on a miss or
+// once the path holds q_len nodes.  The pages' crash came from a walk over
+// cyclic pointers; here every examined node counts against q_len, and pointers
+// are range-checked before use, so the walk ends on any input.
+// One warp per request: the warp stages the request's four arrays in shared
+// memory, lane 0 walks, and the warp writes the padded path back.
+// ---------------------------------------------------------------------------
+constexpr int kAcceptWarps = 4;
+
+__global__ void __launch_bounds__(kAcceptWarps * 32) tree_accept_kernel(
+    const int32_t* __restrict__ node_tokens, const int32_t* __restrict__ target_tokens,
+    const int32_t* __restrict__ next_token, const int32_t* __restrict__ next_sibling, int B,
+    int q_len, int32_t* __restrict__ path, int32_t* __restrict__ accept_len,
+    int32_t* __restrict__ bonus_token, int32_t* __restrict__ status) {
+  __shared__ int32_t s_tok[kAcceptWarps][DDT_MAX_Q_LEN];
+  __shared__ int32_t s_tgt[kAcceptWarps][DDT_MAX_Q_LEN];
+  __shared__ int32_t s_first[kAcceptWarps][DDT_MAX_Q_LEN];
+  __shared__ int32_t s_sib[kAcceptWarps][DDT_MAX_Q_LEN];
+  __shared__ int32_t s_path[kAcceptWarps][DDT_MAX_Q_LEN];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * kAcceptWarps + warp;
+  if (b >= B) return;
+  const int64_t base = static_cast<int64_t>(b) * q_len;
+  for (int k = lane; k < q_len; k += 32) {
+    s_tok[warp][k] = node_tokens[base + k];
+    s_tgt[warp][k] = target_tokens[base + k];
+    s_first[warp][k] = next_token[base + k];
+    s_sib[warp][k] = next_sibling[base + k];
+    s_path[warp][k] = -1;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    int alen = 1, cur = 0, examined = 0, st = DDT_REQ_OK;
+    s_path[warp][0] = 0;
+    while (alen < q_len) {
+      int c = s_first[warp][cur];
+      int found = -1;
+      while (c != -1) {
+        if (c < 0 || c >= q_len) {
+          st = DDT_REQ_BAD_INDEX;
+          break;
+        }
+        if (++examined > q_len) {
+          st = DDT_REQ_WALK_LIMIT;
+          break;
+        }
+        if (s_tok[warp][c] == s_tgt[warp][cur]) {
+          found = c;
+          break;
+        }
+        c = s_sib[warp][c];
+      }
+      if (st != DDT_REQ_OK || found == -1) break;
+      s_path[warp][alen++] = found;
+      cur = found;
+    }
+    accept_len[b] = alen;
+    if (bonus_token) bonus_token[b] = s_tgt[warp][cur];
+    if (status) status[b] = st;
+  }
+  __syncwarp();
+  for (int k = lane; k < q_len; k += 32) path[base + k] = s_path[warp][k];
+}
+
+// ---------------------------------------------------------------------------
+// Compaction.  [Race Conditions] "The Cache Compaction Problem": row P+i takes
+// old row P+keep[i].  A parallel in-place gather races when keep[j] = i' (row
+// i' read by one thread while another writes it); the pages route the gather
+// through scratch buffers.  Here one CTA owns a request: it reads every kept row
+// (latent and rope parts) into shared memory with 16-byte loads, synchronises,
+// and only then writes, so no write can precede a read of the same row — for
+// any path, without scratch memory.  Rows that do not move (keep[i] == i) are
+// not rewritten.
+// ---------------------------------------------------------------------------
+constexpr int kCompactThreads = 256;
+constexpr int kLatVec = DDT_D_LATENT * 2 / 16;  // 16-byte vectors per latent row (64)
+constexpr int kRopeVec = DDT_D_ROPE * 2 / 16;   // per rope row (8)
+constexpr int kRowVec = kLatVec + kRopeVec;
+
+__global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
+    uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
+    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* __restrict__ prefix_lens,
+    const int32_t* __restrict__ path, const int32_t* __restrict__ accept_len, int q_len,
+    int32_t* __restrict__ new_prefix_lens, int32_t* __restrict__ status) {
+  extern __shared__ uint4 s_rows[];  // [alen][kRowVec]
+  __shared__ int32_t s_keep[DDT_MAX_Q_LEN];
+  __shared__ int s_state;  // 0 ok, else status code
+  const int b = blockIdx.x;
+  const int P = prefix_lens[b];
+  const int alen = accept_len[b];
+  if (threadIdx.x == 0) {
+    int st = DDT_REQ_OK;
+    if (alen < 1 || alen > q_len) st = DDT_REQ_BAD_LENGTH;
+    else if (P < 0 || static_cast<int64_t>(P) + q_len > capacity) st = DDT_REQ_BAD_PREFIX;
+    s_state = st;
+  }
+  __syncthreads();
+  if (s_state == DDT_REQ_OK) {
+    int bad = 0;
+    for (int i = threadIdx.x; i < alen; i += kCompactThreads) {
+      const int k = path[static_cast<int64_t>(b) * q_len + i];
+      s_keep[i] = k;
+      bad |= (k < 0 || k >= q_len);
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) s_state = DDT_REQ_BAD_INDEX;
+    __syncthreads();
+  }
+  const int st = s_state;
+  if (st != DDT_REQ_OK) {
+    if (threadIdx.x == 0) {
+      if (status) status[b] = st;
+      if (new_prefix_lens) new_prefix_lens[b] = P;
+    }
+    return;
+  }
+  const uint4* ckv_b = reinterpret_cast<const uint4*>(c_kv + b * ckv_bs);
+  const uint4* kr_b = reinterpret_cast<const uint4*>(k_rope + b * kr_bs);
+  const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;  // row strides in 16-byte vectors
+  const int total = alen * kRowVec;
+  // Phase 1: every moving row into shared memory.
+  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
+    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    if (s_keep[i] == i) continue;
+    const int64_t src_row = P + s_keep[i];
+    s_rows[idx] = (v < kLatVec) ? ckv_b[src_row * ckv_rv + v] : kr_b[src_row * kr_rv + (v - kLatVec)];
+  }
+  __syncthreads();
+  // Phase 2: write rows P .. P+alen-1 (only those that move).
+  uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
+  uint4* kr_w = reinterpret_cast<uint4*>(k_rope + b * kr_bs);
+  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
+    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    if (s_keep[i] == i) continue;
+    const int64_t dst_row = P + i;
+    if (v < kLatVec) ckv_w[dst_row * ckv_rv + v] = s_rows[idx];
+    else kr_w[dst_row * kr_rv + (v - kLatVec)] = s_rows[idx];
+  }
+  if (threadIdx.x == 0) {
+    if (status) status[b] = DDT_REQ_OK;
+    if (new_prefix_lens) new_prefix_lens[b] = P + alen;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+cudaError_t launch_build_mask(const int32_t* parents, int B, int q_len, uint64_t* mask,
+                              int32_t* depth, int32_t* status, cudaStream_t stream) {
+  build_mask_kernel<<<B, 128, 0, stream>>>(parents, q_len, mask, depth, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tree_accept(const int32_t* node_tokens, const int32_t* target_tokens,
+                               const int32_t* next_token, const int32_t* next_sibling, int B,
+                               int q_len, int32_t* path, int32_t* accept_len, int32_t* bonus,
+                               int32_t* status, cudaStream_t stream) {
+  const int grid = (B + kAcceptWarps - 1) / kAcceptWarps;
+  tree_accept_kernel<<<grid, kAcceptWarps * 32, 0, stream>>>(
+      node_tokens, target_tokens, next_token, next_sibling, B, q_len, path, accept_len, bonus,
+      status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_compact(uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs, int64_t ckv_rs,
+                              int64_t kr_bs, int64_t kr_rs, int capacity,
+                              const int32_t* prefix_lens, const int32_t* path,
+                              const int32_t* accept_len, int B, int q_len,
+                              int32_t* new_prefix_lens, int32_t* status, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(q_len) * kRowVec * sizeof(uint4);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kv_compact_kernel),
+                                    static_cast<int>(DDT_MAX_Q_LEN * kRowVec * sizeof(uint4)), 0);
+  if (e != cudaSuccess) return e;
+  kv_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
+      c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, capacity, prefix_lens, path, accept_len, q_len,
+      new_prefix_lens, status);
+  return cudaGetLastError();
+}
+
+}  // namespace ddt

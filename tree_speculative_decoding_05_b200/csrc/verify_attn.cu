@@ -1,0 +1,697 @@
+// verify_attn.cu — tree-verify MLA-absorb attention on sm_100a tensor cores.
+//
+// What it computes (sources: "Race Conditions, Buffer Aliasing, and the
+// Architecture of a Native DDTree Inference Engine", sections "The Mission: A
+// Native DDTree Engine" and "The Cache Compaction Problem"; "The Microsecond
+// Verdict: Validating a DDTree Kernel Fix Under Time Pressure", section "The
+// Timeout That Tells a Story"): for request b with prefix P and tree block at
+// cache rows P .. P+Q-1, every (node i, head h) row attends over the cache rows
+// j < P+Q that it may see (all prefix rows; tree row P+a iff a is i or an
+// ancestor of i) with score scale * ([q_lat|q_rope] . [c_kv|k_rope]) and value
+// c_kv.  The pages' kernel re-read the shared latent cache once per head; here
+// each KV tile is fetched once per pair of CTAs and feeds all 128 query rows
+// (two tree nodes x 64 heads) they hold.
+//
+// Design (one CTA pair = one thread-block cluster of 2 on two SMs):
+//   * 128 query rows per pair, 64 per CTA (one tree node, all 64 heads), as the
+//     M dimension of cta_group::2 tcgen05 MMAs (M = 128).  The accumulator
+//     layout of that shape gives each CTA its 64 rows spread over all 128 TMEM
+//     lanes: lanes 0-63 hold columns [0, N/2) and lanes 64-127 columns [N/2, N).
+//   * S = Q K^T per 128-key tile: 36 MMAs of N = 128, K = 16 (576 = 9 chunks of
+//     64).  Q (64 rows x 576, 72 KB per CTA) stays in shared memory; each CTA
+//     stages its half of the keys (64 keys x 64 dims = 8 KB per stage).
+//   * O += P V per tile: 16 MMAs of N = 256, K = 16 into two fp32 accumulators
+//     covering the 512 latent columns (128 TMEM columns each per CTA).  V is the
+//     same c_kv rows read as an MN-major operand (each CTA stages 128 latent
+//     columns x 32 keys = 8 KB per stage).
+//   * TMEM per CTA: S double buffer (2 x 64 cols) + O (256 cols) of 512.
+//   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
+//     half of one query row), warp 4 TMA producer, warp 5 MMA issuer (the
+//     even CTA of the pair issues for both).
+//   * Online softmax in registers with exp2; the row maximum of the two half
+//     rows is exchanged through shared memory; O is rescaled lazily, only when
+//     the running maximum grows by more than 2^8.
+//   * Long caches: the KV tiles of a request are split into num_splits ranges
+//     handled by different pairs; each writes a normalised partial output and
+//     its log-sum-exp, and a merge kernel combines them.
+//   * Cache rows at or past P+Q (padding, possibly non-finite) are never used:
+//     their scores are masked by index and their V rows are zeroed in shared
+//     memory before the P V product.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "ddt.h"
+#include "ddt_internal.h"
+
+namespace ddt {
+__device__ unsigned int ddt_fault_word = 0;  // bit set, see ddt_fault_flags
+}  // namespace ddt
+
+#include "sm100_ptx.cuh"
+
+namespace ddt {
+
+namespace va {
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr int kStageBytes = 8192;
+constexpr int kStages = 12;
+constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
+constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
+constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
+constexpr int kOffQ = 0;
+constexpr int kOffRing = kOffQ + kQBytes;
+constexpr int kOffP = kOffRing + kStages * kStageBytes;
+constexpr int kOffRedMax = kOffP + 2 * kPBufBytes;     // float[2][128]
+constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
+constexpr int kOffBar = kOffRedL + 128 * 4;
+// barriers: full[kStages], empty[kStages], q_full, s_full[2], p_full[2], o_done, fix, mma_done
+constexpr int kBarFull = 0;
+constexpr int kBarEmpty = kBarFull + kStages;
+constexpr int kBarQ = kBarEmpty + kStages;
+constexpr int kBarS = kBarQ + 1;
+constexpr int kBarP = kBarS + 2;
+constexpr int kBarO = kBarP + 2;
+constexpr int kBarFix = kBarO + 1;
+constexpr int kBarDone = kBarFix + 1;
+constexpr int kNumBars = kBarDone + 1;
+constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmemPtr + 4;
+constexpr int kSmemUsed = kOffAbort + 4;
+constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+constexpr int kTmemCols = 512;
+constexpr int kTmemS = 0;    // S buffers at columns 0 and 64
+constexpr int kTmemO = 128;  // O halves at columns 128 and 256
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+}  // namespace va
+
+struct VerifyParams {
+  const int32_t* prefix_lens;
+  const uint64_t* mask;
+  void* out;
+  float* lse;
+  float* part_o;    // [num_splits][B*Q*64][512], used when num_splits > 1
+  float* part_lse;  // [num_splits][B*Q*64]
+  int32_t* status;
+  int B, Q, capacity, num_splits, n_pairs, out_f32;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+// KV tile range [t0, t1) of split `split` for a cache of T rows.
+__host__ __device__ inline void split_range(int T, int num_splits, int split, int& t0, int& t1) {
+  const int n_tiles = (T + 127) / 128;
+  const int per = (n_tiles + num_splits - 1) / num_splits;
+  t0 = split * per;
+  t1 = t0 + per < n_tiles ? t0 + per : n_tiles;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
+    verify_attn_kernel(const __grid_constant__ CUtensorMap tm_qlat,
+                       const __grid_constant__ CUtensorMap tm_qrope,
+                       const __grid_constant__ CUtensorMap tm_ckv_k,
+                       const __grid_constant__ CUtensorMap tm_ckv_v,
+                       const __grid_constant__ CUtensorMap tm_krope, const VerifyParams p) {
+  using namespace va;
+  const uint32_t rank = cluster_ctarank();
+  const int item = blockIdx.x >> 1;
+  const int per_req = p.n_pairs * p.num_splits;
+  const int b = item / per_req;
+  const int rem = item - b * per_req;
+  const int pair = rem / p.num_splits;
+  const int split = rem - pair * p.num_splits;
+  const int node = 2 * pair + static_cast<int>(rank);
+  const int Q = p.Q;
+  const int P = p.prefix_lens[b];
+
+  // Requests whose tree block would not fit the cache are rejected as a whole;
+  // both CTAs of every pair reach the same decision.
+  const bool bad_prefix = (P < 0) || (static_cast<int64_t>(P) + Q > p.capacity);
+  if (rank == 0 && pair == 0 && split == 0 && threadIdx.x == 0 && p.status)
+    p.status[b] = bad_prefix ? DDT_REQ_BAD_PREFIX : DDT_REQ_OK;
+  if (bad_prefix) return;
+  const int T = P + Q;
+  int t0, t1;
+  split_range(T, p.num_splits, split, t0, t1);
+  if (t0 >= t1) return;  // empty split: the merge skips it
+  const int ntile = t1 - t0;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  const uint32_t sQ = base_addr + kOffQ;
+  const uint32_t sRing = base_addr + kOffRing;
+  const uint32_t sP = base_addr + kOffP;
+  float* red_max = reinterpret_cast<float*>(base + kOffRedMax);
+  float* red_l = reinterpret_cast<float*>(base + kOffRedL);
+  const uint32_t bars = base_addr + kOffBar;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_ptr_smem = reinterpret_cast<uint32_t*>(base + kOffTmemPtr);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarFull + s), 2);   // one arrival per CTA of the pair
+      mbar_init(bar(kBarEmpty + s), 1);  // the MMA issuer's commit
+    }
+    mbar_init(bar(kBarQ), 2);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarS + s), 1);
+      mbar_init(bar(kBarP + s), 2);  // one arrival per CTA of the pair
+    }
+    mbar_init(bar(kBarO), 1);
+    mbar_init(bar(kBarFix), 1);
+    mbar_init(bar(kBarDone), 1);
+    *abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 5) {
+    tmem_alloc<2>(smem_u32(tmem_ptr_smem), kTmemCols);
+    tmem_relinquish<2>();
+  }
+  tc_fence_before_sync();
+  cluster_sync();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_ptr_smem;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t fix_phase = 0;
+    const int key_half = static_cast<int>(rank) * 64;
+    if (lane == 0) {
+      const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
+      mbar_arrive_expect_tx_cluster(qbar, kQBytes);
+      for (int c = 0; c < 8; ++c)
+        tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
+      tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
+    }
+    auto acquire = [&]() { mbar_wait(bar(kBarEmpty + stage), phase ^ 1u, abort_flag); };
+    auto advance = [&]() {
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    };
+    auto produce_k = [&](int tile) {
+      const int key0 = tile * 128 + key_half;
+      for (int c = 0; c < kQChunks; ++c) {
+        acquire();
+        if (lane == 0) {
+          const uint32_t fb = map_to_rank(bar(kBarFull + stage), 0);
+          mbar_arrive_expect_tx_cluster(fb, kStageBytes);
+          const uint32_t dst = sRing + stage * kStageBytes;
+          if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, b);
+          else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, b);
+        }
+        __syncwarp();
+        advance();
+      }
+    };
+    auto produce_v = [&](int tile) {
+      for (int kb = 0; kb < 4; ++kb) {
+        const int key0 = tile * 128 + 32 * kb;
+        const int valid = T - key0;  // rows of this 32-key box that are real cache rows
+        for (int nh = 0; nh < 2; ++nh) {
+          acquire();
+          const int x0 = 256 * nh + 128 * static_cast<int>(rank);
+          const uint32_t dst = sRing + stage * kStageBytes;
+          const uint32_t fb = map_to_rank(bar(kBarFull + stage), 0);
+          if (valid >= 32) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx_cluster(fb, kStageBytes);
+              tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, b);
+              tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, b);
+            }
+            __syncwarp();
+          } else {
+            // Rows at or past P+Q: zero them in shared memory (after loading the
+            // valid rows, if any), then release the stage.
+            if (valid > 0) {
+              if (lane == 0) {
+                mbar_arrive_expect_tx_local(bar(kBarFix), kStageBytes);
+                tma_load_3d(dst, &tm_ckv_v, bar(kBarFix), x0, key0, b);
+                tma_load_3d(dst + 4096, &tm_ckv_v, bar(kBarFix), x0 + 64, key0, b);
+              }
+              mbar_wait(bar(kBarFix), fix_phase, abort_flag);
+              fix_phase ^= 1u;
+            }
+            const int first_bad = valid > 0 ? valid : 0;
+            const int nvec = (32 - first_bad) * 8;  // 16-byte vectors per chunk
+            uint4* s0 = reinterpret_cast<uint4*>(base + kOffRing + stage * kStageBytes);
+            for (int v = lane; v < nvec; v += 32) {
+              s0[first_bad * 8 + v] = make_uint4(0, 0, 0, 0);
+              s0[256 + first_bad * 8 + v] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(fb);
+          }
+          advance();
+        }
+      }
+    };
+    produce_k(t0);
+    for (int jj = 1; jj < ntile; ++jj) {
+      produce_k(t0 + jj);
+      produce_v(t0 + jj - 1);
+    }
+    produce_v(t0 + ntile - 1);
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA
+    if (rank == 0 && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      auto advance = [&]() {
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
+      mbar_wait(bar(kBarQ), 0, abort_flag);
+      tc_fence_after_sync();
+      auto issue_qk = [&](int jj) {
+        const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(jj & 1);
+        for (int c = 0; c < kQChunks; ++c) {
+          mbar_wait(bar(kBarFull + stage), phase, abort_flag);
+          tc_fence_after_sync();
+          const uint32_t a0 = sQ + c * kStageBytes;
+          const uint32_t b0 = sRing + stage * kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
+                           smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
+          mma_commit<2>(bar(kBarEmpty + stage), 0x3);
+          advance();
+        }
+        mma_commit<2>(bar(kBarS + (jj & 1)), 0x3);
+      };
+      auto issue_pv = [&](int jj) {
+        const int pb = jj & 1;
+        mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((jj >> 1) & 1), abort_flag);
+        tc_fence_after_sync();
+        for (int kb = 0; kb < 4; ++kb) {
+          for (int nh = 0; nh < 2; ++nh) {
+            mbar_wait(bar(kBarFull + stage), phase, abort_flag);
+            tc_fence_after_sync();
+            const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
+            const uint32_t a0 = sP + pb * kPBufBytes + (kb >> 1) * kStageBytes + (kb & 1) * 64;
+            const uint32_t b0 = sRing + stage * kStageBytes;
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+              mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
+                             smem_desc_sw128(b0 + 2048 * ks, 4096, 1024), kIdescPV,
+                             !(jj == 0 && kb == 0 && ks == 0));
+            mma_commit<2>(bar(kBarEmpty + stage), 0x3);
+            advance();
+          }
+        }
+        mma_commit<2>(bar(kBarO), 0x3);
+      };
+      issue_qk(0);
+      for (int jj = 1; jj < ntile; ++jj) {
+        issue_qk(jj);
+        issue_pv(jj - 1);
+      }
+      issue_pv(ntile - 1);
+      mma_commit<2>(bar(kBarDone), 0x1);
+      mbar_wait(bar(kBarDone), 0, abort_flag);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------- softmax warps
+    const int t = threadIdx.x;         // TMEM lane
+    const int m = t & 63;              // row within this CTA (head)
+    const int hf = t >> 6;             // which half of the 128-key tile / O columns
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const bool node_valid = node < Q;
+    const int W = (Q + 63) >> 6;
+    uint64_t mw0 = 0, mw1 = 0;
+    if (node_valid) {
+      const uint64_t* mrow = p.mask + (static_cast<int64_t>(b) * Q + node) * W;
+      mw0 = mrow[0];
+      if (W > 1) mw1 = mrow[1];
+    }
+    const uint32_t p_full_leader0 = map_to_rank(bar(kBarP), 0);
+    float m_ref = -INFINITY;
+    float l_sum = 0.f;
+    float m_use = 0.f;
+    for (int jj = 0; jj < ntile; ++jj) {
+      const int tile = t0 + jj;
+      const int sb = jj & 1;
+      mbar_wait(bar(kBarS + sb), static_cast<uint32_t>((jj >> 1) & 1), abort_flag);
+      tc_fence_after_sync();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lane_addr + kTmemS + 64u * sb, r0);
+      tmem_ld32(tmem + lane_addr + kTmemS + 64u * sb + 32u, r1);
+      tmem_wait_ld();
+      float x[64];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = __uint_as_float(r0[c]) * p.scale_log2;
+        x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
+      }
+      const int key0 = tile * 128 + hf * 64;
+      if (key0 + 64 > P) {  // tile reaches into the tree block or past it
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = key0 + c;
+          bool vis = key < P;
+          if (!vis && key < T) {
+            const int a = key - P;
+            const uint64_t w = a < 64 ? mw0 : mw1;
+            vis = (w >> (a & 63)) & 1ull;
+          }
+          if (!vis) x[c] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+      red_max[sb * 128 + t] = mx;
+      named_barrier_sync(1, kSoftmaxThreads);
+      mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]);
+      float factor = 1.f;
+      bool rescale = false;
+      if (m_ref == -INFINITY) {
+        m_ref = mx;  // nothing accumulated yet: adopt the first finite maximum
+      } else if (mx > m_ref + kRescaleLog2) {
+        factor = fast_exp2(m_ref - mx);
+        m_ref = mx;
+        l_sum *= factor;
+        rescale = true;
+      }
+      m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // The row sum takes the bf16-rounded weights, the values the P V product
+      // multiplies, so the normalised weights sum to one exactly.
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float e0 = fast_exp2(x[2 * c] - m_use);
+        const float e1 = fast_exp2(x[2 * c + 1] - m_use);
+        pk[c] = pack_bf16x2(e0, e1);
+        l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+      }
+      // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
+      uint8_t* prow = base + kOffP + sb * kPBufBytes + hf * kStageBytes + m * 128;
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
+      }
+      if (jj > 0) {
+        // PV of the previous tile must be complete before O may be rescaled.
+        mbar_wait(bar(kBarO), static_cast<uint32_t>((jj - 1) & 1), abort_flag);
+        tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+          for (int q = 0; q < 8; ++q) {
+            uint32_t o[32];
+            const uint32_t addr = tmem + lane_addr + kTmemO + 32u * q;
+            tmem_ld32(addr, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+            tmem_st32(addr, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      named_barrier_sync(2, kSoftmaxThreads);
+      if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * sb);
+    }
+    // ------------------------------------------------------------- epilogue
+    mbar_wait(bar(kBarO), static_cast<uint32_t>((ntile - 1) & 1), abort_flag);
+    tc_fence_after_sync();
+    red_l[t] = l_sum;
+    named_barrier_sync(1, kSoftmaxThreads);
+    const float l_row = l_sum + red_l[t ^ 64];
+    const bool empty_row = !(l_row > 0.f);
+    const float inv = empty_row ? 0.f : 1.f / l_row;
+    const float lse_nat = empty_row ? -INFINITY : (m_use + __log2f(l_row)) * kLn2;
+    if (node_valid) {
+      const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
+      const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+#pragma unroll 1
+      for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
+          tmem_wait_ld();
+          const int col = 256 * nh + 128 * hf + 32 * q;
+          if (p.num_splits > 1) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.part_o + (static_cast<int64_t>(split) * rows_total + row) * 512 + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                   __uint_as_float(o[4 * v + 2]) * inv,
+                                   __uint_as_float(o[4 * v + 3]) * inv);
+          } else if (p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                   __uint_as_float(o[4 * v + 2]) * inv,
+                                   __uint_as_float(o[4 * v + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * 512 + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+          }
+        }
+      }
+      if (hf == 0) {
+        if (p.num_splits > 1) p.part_lse[static_cast<int64_t>(split) * rows_total + row] = lse_nat;
+        else if (p.lse) p.lse[row] = lse_nat;
+      }
+    }
+  }
+
+  // All MMAs of the pair are complete here (the softmax warps waited for the
+  // last O commit, the issuer for its final commit); release tensor memory.
+  __syncwarp();
+  tc_fence_before_sync();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after_sync();
+    tmem_dealloc<2>(tmem, kTmemCols);
+  }
+}
+
+// Combine split partials: lse = log sum_s exp(lse_s), out = sum_s exp(lse_s - lse) out_s.
+__global__ void __launch_bounds__(256) verify_merge_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_lse,
+                                                           const int32_t* __restrict__ prefix_lens,
+                                                           void* __restrict__ out, int out_f32,
+                                                           float* __restrict__ lse, int B, int Q,
+                                                           int capacity, int num_splits) {
+  const int64_t rows_total = static_cast<int64_t>(B) * Q * 64;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows_total) return;
+  const int b = static_cast<int>(row / (static_cast<int64_t>(Q) * 64));
+  const int P = prefix_lens[b];
+  if (P < 0 || static_cast<int64_t>(P) + Q > capacity) return;
+  const int T = P + Q;
+  float lmax = -INFINITY;
+  int ns = 0;
+  for (int s = 0; s < num_splits; ++s) {
+    int t0, t1;
+    split_range(T, num_splits, s, t0, t1);
+    if (t0 >= t1) break;
+    ns = s + 1;
+    lmax = fmaxf(lmax, part_lse[s * rows_total + row]);
+  }
+  float acc[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float ls = part_lse[s * rows_total + row];
+    const float w = (ls == -INFINITY) ? 0.f : fast_exp2((ls - lmax) * va::kLog2e);
+    wsum += w;
+    const float4* src = reinterpret_cast<const float4*>(part_o + (s * rows_total + row) * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = src[lane + 32 * k];
+      acc[4 * k] += w * v.x;
+      acc[4 * k + 1] += w * v.y;
+      acc[4 * k + 2] += w * v.z;
+      acc[4 * k + 3] += w * v.w;
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  if (out_f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + row * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      dst[lane + 32 * k] = make_float4(acc[4 * k] * inv, acc[4 * k + 1] * inv, acc[4 * k + 2] * inv,
+                                       acc[4 * k + 3] * inv);
+  } else {
+    uint2* dst = reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + row * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      dst[lane + 32 * k] = make_uint2(pack_bf16x2(acc[4 * k] * inv, acc[4 * k + 1] * inv),
+                                      pack_bf16x2(acc[4 * k + 2] * inv, acc[4 * k + 3] * inv));
+  }
+  if (lse && lane == 0) lse[row] = (wsum > 0.f) ? lmax + __logf(wsum) : -INFINITY;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 map: dims {d0 (contiguous), d1, d2}, byte strides of d1 and d2, box
+// {64, box1, 1}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {64, box1, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int verify_num_splits(const ddt_attn_args& a, int sm_count) {
+  if (a.num_splits > 0) return a.num_splits;
+  const int n_pairs = (a.q_len + 1) / 2;
+  const int64_t items = static_cast<int64_t>(a.B) * n_pairs;
+  const int pairs_avail = sm_count / 2 > 0 ? sm_count / 2 : 1;
+  const int max_tiles = (a.max_prefix + a.q_len + 127) / 128;
+  // Score = wave efficiency x share of a work item spent on KV tiles (each item
+  // also pays about 1.5 tiles of fixed cost: set-up, Q load, pipeline fill).
+  auto score = [&](int s) {
+    const int64_t n = items * s;
+    const int64_t waves = (n + pairs_avail - 1) / pairs_avail;
+    const double eff = static_cast<double>(n) / static_cast<double>(waves * pairs_avail);
+    const int per = (max_tiles + s - 1) / s;
+    return eff * per / (per + 1.5);
+  };
+  int best = 1;
+  double best_score = score(1);
+  for (int s = 2; s <= 32 && s <= max_tiles; ++s) {
+    const double sc = score(s);
+    if (sc > best_score * 1.02) {
+      best = s;
+      best_score = sc;
+    }
+  }
+  return best;
+}
+
+size_t verify_workspace_bytes(const ddt_attn_args& a, int num_splits) {
+  if (num_splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(a.B) * a.q_len * 64;
+  return static_cast<size_t>(num_splits) * rows * (512 + 1) * sizeof(float);
+}
+
+ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* part_o,
+                              float* part_lse, cudaStream_t stream) {
+  using namespace va;
+  CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope;
+  const uint64_t rows_q = static_cast<uint64_t>(a.q_len) * 64;
+  const uint64_t B = static_cast<uint64_t>(a.B);
+  const uint64_t cap = static_cast<uint64_t>(a.capacity);
+  bool ok = make_map(&m_qlat, a.q_lat, 512, rows_q, B, 512 * 2, rows_q * 512 * 2, 64) &&
+            make_map(&m_qrope, a.q_rope, 64, rows_q, B, 64 * 2, rows_q * 64 * 2, 64) &&
+            make_map(&m_ckv_k, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 64) &&
+            make_map(&m_ckv_v, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 32) &&
+            make_map(&m_krope, a.k_rope, 64, cap, B, a.kr_row_stride * 2, a.kr_batch_stride * 2, 64);
+  if (!ok) return DDT_ERR_INVALID_ARG;
+  if (ensure_smem_limit(reinterpret_cast<const void*>(verify_attn_kernel), kSmemBytes, 1) !=
+      cudaSuccess)
+    return DDT_ERR_CUDA;
+  VerifyParams p;
+  p.prefix_lens = a.prefix_lens;
+  p.mask = a.mask;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.status = a.status;
+  p.B = a.B;
+  p.Q = a.q_len;
+  p.capacity = a.capacity;
+  p.num_splits = num_splits;
+  p.n_pairs = (a.q_len + 1) / 2;
+  p.out_f32 = a.out_dtype == DDT_F32;
+  p.scale_log2 = a.softmax_scale * kLog2e;
+  const int64_t grid = 2ll * a.B * p.n_pairs * num_splits;
+  if (grid > 0x7fffffffll) return DDT_ERR_UNSUPPORTED;
+  verify_attn_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
+      m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, p);
+  if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
+  if (num_splits > 1) {
+    const int64_t rows = static_cast<int64_t>(a.B) * a.q_len * 64;
+    verify_merge_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        part_o, part_lse, a.prefix_lens, a.out, p.out_f32, a.lse, a.B, a.q_len, a.capacity,
+        num_splits);
+    if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
+  }
+  return DDT_OK;
+}
+
+}  // namespace ddt
+
+// Diagnostic read of the library's device fault word (synchronises the device).
+extern "C" ddt_status ddt_fault_flags(uint32_t* flags, int32_t reset) {
+  if (!flags) return DDT_ERR_INVALID_ARG;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ddt::ddt_fault_word, sizeof v) != cudaSuccess) return DDT_ERR_CUDA;
+  *flags = v;
+  if (reset) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(ddt::ddt_fault_word, &zero, sizeof zero) != cudaSuccess)
+      return DDT_ERR_CUDA;
+  }
+  return DDT_OK;
+}
