@@ -26,17 +26,18 @@
 //     columns x 32 keys = 8 KB per stage).
 //   * TMEM per CTA: S double buffer (2 x 64 cols) + O (256 cols) of 512.
 //   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
-//     half of one query row), warp 4 TMA producer, warp 5 MMA issuer (the
-//     even CTA of the pair issues for both).
+//     half of one query row); warps 4 and 6 TMA producers of the K ring and
+//     the V ring; warps 5 and 7 issue the S = Q K^T and the O += P V MMAs (the
+//     even CTA of the pair issues for both).  Two issuing threads keep the
+//     tensor core fed while either one waits on a barrier or commits a stage.
 //   * Online softmax in registers with exp2; the row maximum of the two half
 //     rows is exchanged through shared memory; O is rescaled lazily, only when
 //     the running maximum grows by more than 2^8.
 //   * Long caches: the KV tiles of a request are split into num_splits ranges
 //     handled by different pairs; each writes a normalised partial output and
 //     its log-sum-exp, and a merge kernel combines them.
-//   * Cache rows at or past P+Q (padding, possibly non-finite) are never used:
-//     their scores are masked by index and their V rows are zeroed in shared
-//     memory before the P V product.
+//   * Cache rows at or past P+Q (padding, possibly non-finite) are never
+//     loaded: the last KV tile of a request ends exactly at row P+Q.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -56,29 +57,34 @@ __device__ unsigned int ddt_fault_word = 0;  // bit set, see ddt_fault_flags
 namespace ddt {
 
 namespace va {
-constexpr int kThreads = 192;
+constexpr int kThreads = 256;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kStageBytes = 8192;
-constexpr int kStages = 12;
+constexpr int kKStages = 8;                        // K ring (feeds S = Q K^T)
+constexpr int kVStages = 6;                        // V ring (feeds O += P V)
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
 constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kStageBytes;
+constexpr int kOffKRing = kOffQ + kQBytes;
+constexpr int kOffVRing = kOffKRing + kKStages * kStageBytes;
+constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffRedMax = kOffP + 2 * kPBufBytes;     // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
 constexpr int kOffBar = kOffRedL + 128 * 4;
-// barriers: full[kStages], empty[kStages], q_full, s_full[2], p_full[2], o_done, fix, mma_done
-constexpr int kBarFull = 0;
-constexpr int kBarEmpty = kBarFull + kStages;
-constexpr int kBarQ = kBarEmpty + kStages;
+// barriers: K ring full/empty, V ring full/empty, q_full, s_full[2], p_full[2],
+// o_done, and one "all issued MMAs done" barrier per issuing thread.
+constexpr int kBarKFull = 0;
+constexpr int kBarKEmpty = kBarKFull + kKStages;
+constexpr int kBarVFull = kBarKEmpty + kKStages;
+constexpr int kBarVEmpty = kBarVFull + kVStages;
+constexpr int kBarQ = kBarVEmpty + kVStages;
 constexpr int kBarS = kBarQ + 1;
 constexpr int kBarP = kBarS + 2;
 constexpr int kBarO = kBarP + 2;
-constexpr int kBarFix = kBarO + 1;
-constexpr int kBarDone = kBarFix + 1;
-constexpr int kNumBars = kBarDone + 1;
+constexpr int kBarQKDone = kBarO + 1;
+constexpr int kBarPVDone = kBarQKDone + 1;
+constexpr int kNumBars = kBarPVDone + 1;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemUsed = kOffAbort + 4;
@@ -144,13 +150,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   split_range(T, p.num_splits, split, t0, t1);
   if (t0 >= t1) return;  // empty split: the merge skips it
   const int ntile = t1 - t0;
+  // First cache row of KV tile t.  The request's last tile is shifted to end at
+  // row T, so no load ever reaches the rows past the tree block (padding that
+  // may hold anything); its overlap with the previous tile is masked, and rows
+  // below 0 (T < 128) read as zeros.
+  const int last_tile = (T + 127) / 128 - 1;
+  auto tile_start = [&](int t) -> int { return t == last_tile ? T - 128 : 128 * t; };
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
   const uint32_t sQ = base_addr + kOffQ;
-  const uint32_t sRing = base_addr + kOffRing;
+  const uint32_t sKRing = base_addr + kOffKRing;
+  const uint32_t sVRing = base_addr + kOffVRing;
   const uint32_t sP = base_addr + kOffP;
   float* red_max = reinterpret_cast<float*>(base + kOffRedMax);
   float* red_l = reinterpret_cast<float*>(base + kOffRedL);
@@ -163,18 +176,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 2);   // one arrival per CTA of the pair
-      mbar_init(bar(kBarEmpty + s), 1);  // the MMA issuer's commit
+    // Stage and Q barriers: one arrival (the even CTA's producer, expecting the
+    // bytes of both CTAs); the odd CTA's loads only add completed bytes.
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);  // the issuing thread's commit
     }
-    mbar_init(bar(kBarQ), 2);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    mbar_init(bar(kBarQ), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarS + s), 1);
       mbar_init(bar(kBarP + s), 2);  // one arrival per CTA of the pair
     }
     mbar_init(bar(kBarO), 1);
-    mbar_init(bar(kBarFix), 1);
-    mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarQKDone), 1);
+    mbar_init(bar(kBarPVDone), 1);
     *abort_flag = 0;
     fence_mbar_init_cluster();
   }
@@ -187,149 +206,122 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_ptr_smem;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ TMA
+  // Ring helper: a stage index and phase bit advancing over `n` stages.
+  struct Ring {
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t fix_phase = 0;
-    const int key_half = static_cast<int>(rank) * 64;
-    if (lane == 0) {
-      const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
-      mbar_arrive_expect_tx_cluster(qbar, kQBytes);
-      for (int c = 0; c < 8; ++c)
-        tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
-      tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
-    }
-    auto acquire = [&]() { mbar_wait(bar(kBarEmpty + stage), phase ^ 1u, abort_flag); };
-    auto advance = [&]() {
-      if (++stage == kStages) {
+    __device__ void advance(int n) {
+      if (++stage == n) {
         stage = 0;
         phase ^= 1u;
       }
-    };
-    auto produce_k = [&](int tile) {
-      const int key0 = tile * 128 + key_half;
-      for (int c = 0; c < kQChunks; ++c) {
-        acquire();
-        if (lane == 0) {
-          const uint32_t fb = map_to_rank(bar(kBarFull + stage), 0);
-          mbar_arrive_expect_tx_cluster(fb, kStageBytes);
-          const uint32_t dst = sRing + stage * kStageBytes;
+    }
+  };
+  const bool leader = rank == 0;
+
+  if (warp == 4) {
+    // ---------------------------------------------------- TMA: Q and K ring
+    // Lane 0 issues.  Only the even CTA arrives on the stage barriers (with the
+    // byte count of both CTAs); both CTAs' loads complete bytes on them.
+    if (lane == 0) {
+      const int key_half = static_cast<int>(rank) * 64;
+      const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
+      if (leader) mbar_arrive_expect_tx_local(bar(kBarQ), 2 * kQBytes);
+      for (int c = 0; c < 8; ++c)
+        tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
+      tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
+      Ring r;
+      for (int jj = 0; jj < ntile; ++jj) {
+        const int key0 = tile_start(t0 + jj) + key_half;
+        for (int c = 0; c < kQChunks; ++c) {
+          mbar_wait(bar(kBarKEmpty + r.stage), r.phase ^ 1u, abort_flag);
+          if (leader) mbar_arrive_expect_tx_local(bar(kBarKFull + r.stage), 2 * kStageBytes);
+          const uint32_t fb = map_to_rank(bar(kBarKFull + r.stage), 0);
+          const uint32_t dst = sKRing + r.stage * kStageBytes;
           if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, b);
           else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, b);
-        }
-        __syncwarp();
-        advance();
-      }
-    };
-    auto produce_v = [&](int tile) {
-      for (int kb = 0; kb < 4; ++kb) {
-        const int key0 = tile * 128 + 32 * kb;
-        const int valid = T - key0;  // rows of this 32-key box that are real cache rows
-        for (int nh = 0; nh < 2; ++nh) {
-          acquire();
-          const int x0 = 256 * nh + 128 * static_cast<int>(rank);
-          const uint32_t dst = sRing + stage * kStageBytes;
-          const uint32_t fb = map_to_rank(bar(kBarFull + stage), 0);
-          if (valid >= 32) {
-            if (lane == 0) {
-              mbar_arrive_expect_tx_cluster(fb, kStageBytes);
-              tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, b);
-              tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, b);
-            }
-            __syncwarp();
-          } else {
-            // Rows at or past P+Q: zero them in shared memory (after loading the
-            // valid rows, if any), then release the stage.
-            if (valid > 0) {
-              if (lane == 0) {
-                mbar_arrive_expect_tx_local(bar(kBarFix), kStageBytes);
-                tma_load_3d(dst, &tm_ckv_v, bar(kBarFix), x0, key0, b);
-                tma_load_3d(dst + 4096, &tm_ckv_v, bar(kBarFix), x0 + 64, key0, b);
-              }
-              mbar_wait(bar(kBarFix), fix_phase, abort_flag);
-              fix_phase ^= 1u;
-            }
-            const int first_bad = valid > 0 ? valid : 0;
-            const int nvec = (32 - first_bad) * 8;  // 16-byte vectors per chunk
-            uint4* s0 = reinterpret_cast<uint4*>(base + kOffRing + stage * kStageBytes);
-            for (int v = lane; v < nvec; v += 32) {
-              s0[first_bad * 8 + v] = make_uint4(0, 0, 0, 0);
-              s0[256 + first_bad * 8 + v] = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(fb);
-          }
-          advance();
+          r.advance(kKStages);
         }
       }
-    };
-    produce_k(t0);
-    for (int jj = 1; jj < ntile; ++jj) {
-      produce_k(t0 + jj);
-      produce_v(t0 + jj - 1);
     }
-    produce_v(t0 + ntile - 1);
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA
-    if (rank == 0 && lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      auto advance = [&]() {
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1u;
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ TMA: V ring
+    if (lane == 0) {
+      Ring r;
+      for (int jj = 0; jj < ntile; ++jj) {
+        for (int kb = 0; kb < 4; ++kb) {
+          const int key0 = tile_start(t0 + jj) + 32 * kb;
+          for (int nh = 0; nh < 2; ++nh) {
+            mbar_wait(bar(kBarVEmpty + r.stage), r.phase ^ 1u, abort_flag);
+            if (leader) mbar_arrive_expect_tx_local(bar(kBarVFull + r.stage), 2 * kStageBytes);
+            const uint32_t fb = map_to_rank(bar(kBarVFull + r.stage), 0);
+            const int x0 = 256 * nh + 128 * static_cast<int>(rank);
+            const uint32_t dst = sVRing + r.stage * kStageBytes;
+            tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, b);
+            tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, b);
+            r.advance(kVStages);
+          }
         }
-      };
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // -------------------------------------------------------- MMA: S = Q K^T
+    if (leader && lane == 0) {
+      Ring r;
       mbar_wait(bar(kBarQ), 0, abort_flag);
-      tc_fence_after_sync();
-      auto issue_qk = [&](int jj) {
+      for (int jj = 0; jj < ntile; ++jj) {
+        if (jj >= 2) {
+          // S buffer jj&1 is free once the softmax of tile jj-2 released its P.
+          mbar_wait(bar(kBarP + (jj & 1)), static_cast<uint32_t>(((jj - 2) >> 1) & 1), abort_flag);
+          tc_fence_after_sync();
+        }
         const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(jj & 1);
         for (int c = 0; c < kQChunks; ++c) {
-          mbar_wait(bar(kBarFull + stage), phase, abort_flag);
-          tc_fence_after_sync();
+          mbar_wait(bar(kBarKFull + r.stage), r.phase, abort_flag);
           const uint32_t a0 = sQ + c * kStageBytes;
-          const uint32_t b0 = sRing + stage * kStageBytes;
+          const uint32_t b0 = sKRing + r.stage * kStageBytes;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
                            smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
-          mma_commit<2>(bar(kBarEmpty + stage), 0x3);
-          advance();
+          mma_commit<2>(bar(kBarKEmpty + r.stage), 0x3);
+          r.advance(kKStages);
         }
         mma_commit<2>(bar(kBarS + (jj & 1)), 0x3);
-      };
-      auto issue_pv = [&](int jj) {
+      }
+      mma_commit<2>(bar(kBarQKDone), 0x1);
+      mbar_wait(bar(kBarQKDone), 0, abort_flag);
+    }
+    __syncwarp();
+  } else if (warp == 7) {
+    // ------------------------------------------------------- MMA: O += P V
+    if (leader && lane == 0) {
+      Ring r;
+      for (int jj = 0; jj < ntile; ++jj) {
         const int pb = jj & 1;
         mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((jj >> 1) & 1), abort_flag);
         tc_fence_after_sync();
         for (int kb = 0; kb < 4; ++kb) {
           for (int nh = 0; nh < 2; ++nh) {
-            mbar_wait(bar(kBarFull + stage), phase, abort_flag);
-            tc_fence_after_sync();
+            mbar_wait(bar(kBarVFull + r.stage), r.phase, abort_flag);
             const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
             const uint32_t a0 = sP + pb * kPBufBytes + (kb >> 1) * kStageBytes + (kb & 1) * 64;
-            const uint32_t b0 = sRing + stage * kStageBytes;
+            const uint32_t b0 = sVRing + r.stage * kStageBytes;
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks)
               mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
                              smem_desc_sw128(b0 + 2048 * ks, 4096, 1024), kIdescPV,
                              !(jj == 0 && kb == 0 && ks == 0));
-            mma_commit<2>(bar(kBarEmpty + stage), 0x3);
-            advance();
+            mma_commit<2>(bar(kBarVEmpty + r.stage), 0x3);
+            r.advance(kVStages);
           }
         }
         mma_commit<2>(bar(kBarO), 0x3);
-      };
-      issue_qk(0);
-      for (int jj = 1; jj < ntile; ++jj) {
-        issue_qk(jj);
-        issue_pv(jj - 1);
       }
-      issue_pv(ntile - 1);
-      mma_commit<2>(bar(kBarDone), 0x1);
-      mbar_wait(bar(kBarDone), 0, abort_flag);
+      mma_commit<2>(bar(kBarPVDone), 0x1);
+      mbar_wait(bar(kBarPVDone), 0, abort_flag);
     }
     __syncwarp();
   } else {
@@ -365,8 +357,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         x[c] = __uint_as_float(r0[c]) * p.scale_log2;
         x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
       }
-      const int key0 = tile * 128 + hf * 64;
-      if (key0 + 64 > P) {  // tile reaches into the tree block or past it
+      const int key0 = tile_start(tile) + hf * 64;
+      const int lo = tile * 128;  // keys below lo belong to the previous tile
+      if (key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = key0 + c;
@@ -376,6 +369,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
             const uint64_t w = a < 64 ? mw0 : mw1;
             vis = (w >> (a & 63)) & 1ull;
           }
+          if (key < lo) vis = false;
           if (!vis) x[c] = -INFINITY;
         }
       }
