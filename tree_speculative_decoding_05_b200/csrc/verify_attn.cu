@@ -26,10 +26,11 @@
 //     columns x 32 keys = 8 KB per stage).
 //   * TMEM per CTA: S double buffer (2 x 64 cols) + O (256 cols) of 512.
 //   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
-//     half of one query row); warps 4 and 6 TMA producers of the K ring and
-//     the V ring; warps 5 and 7 issue the S = Q K^T and the O += P V MMAs (the
-//     even CTA of the pair issues for both).  Two issuing threads keep the
-//     tensor core fed while either one waits on a barrier or commits a stage.
+//     half of one query row); warps 4 and 8 TMA producers of the K rings of
+//     even and odd tiles, warp 6 the producer of the V ring; warps 5 and 9
+//     issue S = Q K^T for even and odd tiles and warp 7 issues O += P V (the
+//     even CTA of the pair issues for both).  Three issuing threads keep the
+//     tensor core fed while each waits on barriers or commits stages.
 //   * Online softmax in registers with exp2; the row maximum of the two half
 //     rows is exchanged through shared memory; O is rescaled lazily, only when
 //     the running maximum grows by more than 2^8.
@@ -57,33 +58,34 @@ __device__ unsigned int ddt_fault_word = 0;  // bit set, see ddt_fault_flags
 namespace ddt {
 
 namespace va {
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kStageBytes = 8192;
-constexpr int kKStages = 8;                        // K ring (feeds S = Q K^T)
+constexpr int kKStages = 4;                        // each of the two K rings (even / odd tiles)
 constexpr int kVStages = 6;                        // V ring (feeds O += P V)
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
 constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
 constexpr int kOffQ = 0;
-constexpr int kOffKRing = kOffQ + kQBytes;
-constexpr int kOffVRing = kOffKRing + kKStages * kStageBytes;
+constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
+constexpr int kOffVRing = kOffKRing + 2 * kKStages * kStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffRedMax = kOffP + 2 * kPBufBytes;     // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
 constexpr int kOffBar = kOffRedL + 128 * 4;
-// barriers: K ring full/empty, V ring full/empty, q_full, s_full[2], p_full[2],
-// o_done, and one "all issued MMAs done" barrier per issuing thread.
+// barriers: two K rings' full/empty (ring g at offset g * kKStages), V ring
+// full/empty, q_full, s_full[2], p_full[2], o_done, and one "all issued MMAs
+// done" barrier per issuing thread (two S issuers, one O issuer).
 constexpr int kBarKFull = 0;
-constexpr int kBarKEmpty = kBarKFull + kKStages;
-constexpr int kBarVFull = kBarKEmpty + kKStages;
+constexpr int kBarKEmpty = kBarKFull + 2 * kKStages;
+constexpr int kBarVFull = kBarKEmpty + 2 * kKStages;
 constexpr int kBarVEmpty = kBarVFull + kVStages;
 constexpr int kBarQ = kBarVEmpty + kVStages;
 constexpr int kBarS = kBarQ + 1;
 constexpr int kBarP = kBarS + 2;
 constexpr int kBarO = kBarP + 2;
-constexpr int kBarQKDone = kBarO + 1;
-constexpr int kBarPVDone = kBarQKDone + 1;
+constexpr int kBarQKDone = kBarO + 1;      // two: one per S issuer
+constexpr int kBarPVDone = kBarQKDone + 2;
 constexpr int kNumBars = kBarPVDone + 1;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
@@ -178,7 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   if (threadIdx.x == 0) {
     // Stage and Q barriers: one arrival (the even CTA's producer, expecting the
     // bytes of both CTAs); the odd CTA's loads only add completed bytes.
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < 2 * kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);  // the issuing thread's commit
     }
@@ -192,7 +194,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_init(bar(kBarP + s), 2);  // one arrival per CTA of the pair
     }
     mbar_init(bar(kBarO), 1);
-    mbar_init(bar(kBarQKDone), 1);
+    mbar_init(bar(kBarQKDone + 0), 1);
+    mbar_init(bar(kBarQKDone + 1), 1);
     mbar_init(bar(kBarPVDone), 1);
     *abort_flag = 0;
     fence_mbar_init_cluster();
@@ -219,25 +222,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   };
   const bool leader = rank == 0;
 
-  if (warp == 4) {
-    // ---------------------------------------------------- TMA: Q and K ring
-    // Lane 0 issues.  Only the even CTA arrives on the stage barriers (with the
+  if (warp == 4 || warp == 8) {
+    // ---------------------------------------------- TMA: Q and the K rings
+    // Lane 0 issues; warp 4 loads Q and the K stages of even tiles, warp 8 those
+    // of odd tiles.  Only the even CTA arrives on the stage barriers (with the
     // byte count of both CTAs); both CTAs' loads complete bytes on them.
     if (lane == 0) {
+      const int g = warp == 4 ? 0 : 1;
       const int key_half = static_cast<int>(rank) * 64;
-      const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
-      if (leader) mbar_arrive_expect_tx_local(bar(kBarQ), 2 * kQBytes);
-      for (int c = 0; c < 8; ++c)
-        tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
-      tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
+      if (g == 0) {
+        const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
+        if (leader) mbar_arrive_expect_tx_local(bar(kBarQ), 2 * kQBytes);
+        for (int c = 0; c < 8; ++c)
+          tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
+        tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
+      }
+      const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
+      const uint32_t ring = sKRing + g * kKStages * kStageBytes;
       Ring r;
-      for (int jj = 0; jj < ntile; ++jj) {
+      for (int jj = g; jj < ntile; jj += 2) {
         const int key0 = tile_start(t0 + jj) + key_half;
         for (int c = 0; c < kQChunks; ++c) {
-          mbar_wait(bar(kBarKEmpty + r.stage), r.phase ^ 1u, abort_flag);
-          if (leader) mbar_arrive_expect_tx_local(bar(kBarKFull + r.stage), 2 * kStageBytes);
-          const uint32_t fb = map_to_rank(bar(kBarKFull + r.stage), 0);
-          const uint32_t dst = sKRing + r.stage * kStageBytes;
+          mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
+          if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kStageBytes);
+          const uint32_t fb = map_to_rank(bar(full0 + r.stage), 0);
+          const uint32_t dst = ring + r.stage * kStageBytes;
           if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, b);
           else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, b);
           r.advance(kKStages);
@@ -266,33 +275,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 5 || warp == 9) {
     // -------------------------------------------------------- MMA: S = Q K^T
+    // Warp 5 issues even tiles into S buffer 0, warp 9 odd tiles into buffer 1.
     if (leader && lane == 0) {
+      const int g = warp == 5 ? 0 : 1;
+      const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
+      const uint32_t ring = sKRing + g * kKStages * kStageBytes;
+      const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(g);
       Ring r;
       mbar_wait(bar(kBarQ), 0, abort_flag);
-      for (int jj = 0; jj < ntile; ++jj) {
+      for (int jj = g; jj < ntile; jj += 2) {
         if (jj >= 2) {
-          // S buffer jj&1 is free once the softmax of tile jj-2 released its P.
-          mbar_wait(bar(kBarP + (jj & 1)), static_cast<uint32_t>(((jj - 2) >> 1) & 1), abort_flag);
+          // S buffer g is free once the softmax of tile jj-2 released its P.
+          mbar_wait(bar(kBarP + g), static_cast<uint32_t>(((jj - 2) >> 1) & 1), abort_flag);
           tc_fence_after_sync();
         }
-        const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(jj & 1);
         for (int c = 0; c < kQChunks; ++c) {
-          mbar_wait(bar(kBarKFull + r.stage), r.phase, abort_flag);
+          mbar_wait(bar(full0 + r.stage), r.phase, abort_flag);
           const uint32_t a0 = sQ + c * kStageBytes;
-          const uint32_t b0 = sKRing + r.stage * kStageBytes;
+          const uint32_t b0 = ring + r.stage * kStageBytes;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
                            smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
-          mma_commit<2>(bar(kBarKEmpty + r.stage), 0x3);
+          mma_commit<2>(bar(empty0 + r.stage), 0x3);
           r.advance(kKStages);
         }
-        mma_commit<2>(bar(kBarS + (jj & 1)), 0x3);
+        mma_commit<2>(bar(kBarS + g), 0x3);
       }
-      mma_commit<2>(bar(kBarQKDone), 0x1);
-      mbar_wait(bar(kBarQKDone), 0, abort_flag);
+      mma_commit<2>(bar(kBarQKDone + g), 0x1);
+      mbar_wait(bar(kBarQKDone + g), 0, abort_flag);
     }
     __syncwarp();
   } else if (warp == 7) {
