@@ -176,6 +176,33 @@ DDT_API int32_t ddt_verify_attn_num_splits(const ddt_attn_args* args);
 
 DDT_API ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t stream);
 
+/* ddt_verify_attn for callers that cannot allocate device memory.
+ *
+ * The pages describe no counterpart of this call; it exists for users of the
+ * library.  Some callers may not call cudaMalloc at all: a plugin inside a host
+ * framework that owns all device memory after start-up, or a latency-critical
+ * decode loop that cannot take the device synchronisation an allocation may
+ * cause.  Such callers cannot hand ddt_verify_attn the workspace its split-KV
+ * path needs.  This call computes exactly what ddt_verify_attn computes, with
+ * args->workspace and args->workspace_bytes ignored: split partials go to a
+ * fixed scratch array inside the library (ddt_verify_attn_noalloc_scratch_bytes()
+ * bytes, 32 MiB, held on every GPU that loads the library until the process
+ * exits).  It allocates nothing.
+ *   - The first call on a device looks the array's address up (this may load
+ *     the library's device code on that device); make it before any stream
+ *     capture on that device.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that overlap on
+ *     the GPU race on it: order them (one stream, or events).
+ *   - num_splits = 0 picks the largest useful split count whose partials fit
+ *     the array (a single split needs none).  A forced num_splits whose
+ *     partials do not fit is rejected with DDT_ERR_UNSUPPORTED before any
+ *     launch.  Other errors are those of ddt_verify_attn. */
+DDT_API ddt_status ddt_verify_attn_noalloc(const ddt_attn_args* args, ddt_stream_t stream);
+
+/* Size in bytes of the scratch array used by ddt_verify_attn_noalloc. */
+DDT_API size_t ddt_verify_attn_noalloc_scratch_bytes(void);
+
 /* ------------------------------------------------------------------------ */
 /* ddt_tree_accept                                                          */
 /* ------------------------------------------------------------------------ */
