@@ -102,6 +102,33 @@ def measured_peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def measured_traffic(config_idx: int):
+    """DRAM bytes per verify launch from the committed ncu summary of the default
+    workload, or None when the kernel source changed since that capture."""
+    import hashlib
+    if config_idx != 2:
+        return None
+    path = os.path.join(ROOT, "profiles", "verify_attn_config2.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        line = line.strip()
+        for key in ("traffic_bytes_per_launch:", "kernel_source_sha256:"):
+            if line.startswith(key):
+                vals[key] = line.split(":", 1)[1].strip()
+    csrc = os.path.join(ROOT, "tree_speculative_decoding_05_b200", "csrc")
+    src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("verify_attn.cu", "sm100_ptx.cuh"))
+    if vals.get("kernel_source_sha256:") != hashlib.sha256(src).hexdigest():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch:"])
+    except (KeyError, ValueError):
+        return None
+
+
 class ClockSampler:
     """Samples SM clocks and throttle reasons with nvidia-smi while running."""
 
@@ -348,19 +375,26 @@ def main(argv=None) -> int:
     stream = torch.cuda.current_stream(device)
 
     def step(ev=None):
-        ddt.build_mask(d["parents"], mask=mask, depth=depth, status=mstatus)
+        # ev: five events bracketing mask | verify | accept | compact
         if ev is not None:
             ev[0].record(stream)
+        ddt.build_mask(d["parents"], mask=mask, depth=depth, status=mstatus)
+        if ev is not None:
+            ev[1].record(stream)
         ddt.verify_attn(d["q_lat"], d["q_rope"], d["c_kv"], d["k_rope"], d["prefix"], mask,
                         w.softmax_scale, max_prefix=max_prefix, out=out, lse=lse,
                         workspace=workspace if ws_bytes else None, status=vstatus)
         if ev is not None:
-            ev[1].record(stream)
+            ev[2].record(stream)
         ddt.tree_accept(d["node_tokens"], d["target_tokens"], d["next_token"],
                         d["next_sibling"], path=path, accept_len=alen, bonus=bonus,
                         status=astatus)
+        if ev is not None:
+            ev[3].record(stream)
         ddt.kv_compact(d["c_kv"], d["k_rope"], d["prefix"], path, alen, new_prefix_lens=newp,
                        status=cstatus)
+        if ev is not None:
+            ev[4].record(stream)
 
     launches_per_step = 4 + (1 if splits > 1 else 0)
     ddt.fault_flags(reset=True)
@@ -369,8 +403,7 @@ def main(argv=None) -> int:
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(physical_gpu_index(local)) as clocks:
         torch.cuda.synchronize()
@@ -382,14 +415,21 @@ def main(argv=None) -> int:
     if world > 1:
         dist.barrier()
     step_ms = t_start.elapsed_time(t_end) / args.steps
-    verify_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    call_ms = [sum(e[k].elapsed_time(e[k + 1]) for e in evs) / args.steps for k in range(4)]
+    verify_ms = call_ms[1]
+    # Compaction bytes moved: each accepted row that moves is read and written
+    # once (latent + rope = 1152 B).
+    path_h, alen_h = path.cpu().numpy(), alen.cpu().numpy()
+    moved = sum(int((path_h[b, :alen_h[b]] != np.arange(alen_h[b])).sum()) for b in range(B))
+    compact_bytes = 2.0 * moved * (DL + DR) * 2
     faults = ddt.fault_flags(reset=True)
     statuses_ok = all(int(s.max()) == 0 for s in (mstatus, vstatus, astatus, cstatus))
 
     flops_local = verify_flops(w.prefix_lens, w.parents)
     bytes_local = verify_bytes(w.prefix_lens, Q, 4 if out_dtype == torch.float32 else 2,
                                w.want_lse)
-    step_ms_max, verify_ms_max = reduce_max([step_ms, verify_ms], world, device)
+    step_ms_max, verify_ms_max, mask_ms_max, accept_ms_max, compact_ms_max = reduce_max(
+        [step_ms, verify_ms, call_ms[0], call_ms[2], call_ms[3]], world, device)
     flops_total = reduce_sum([flops_local], world, device)[0]
 
     # ---- end to end through the public API with host buffers ---------------
@@ -477,10 +517,13 @@ def main(argv=None) -> int:
                              "no flush" % (w.c_kv.nbytes / 1e6 + w.k_rope.nbytes / 1e6,
                                            (w.q_lat.nbytes + w.q_rope.nbytes) / 1e6)},
             "verify_us_per_call": verify_ms_max * 1e3,
+            "calls_us": {"build_mask": mask_ms_max * 1e3, "verify_attn": verify_ms_max * 1e3,
+                         "tree_accept": accept_ms_max * 1e3, "kv_compact": compact_ms_max * 1e3},
+            "kv_compact_gbs": compact_bytes / (compact_ms_max * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} {'sustained' if use_sustained else 'burst'} bf16",
-                         "traffic": None,
+                         "traffic": measured_traffic(args.config),
                          "algorithmic_bytes": bytes_local,
                          "kernel": "verify_attn_kernel"},
             "cpu_baseline": cpu,

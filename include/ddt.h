@@ -168,10 +168,13 @@ typedef struct ddt_attn_args {
   int32_t* status;    /* int32 [B] or NULL: DDT_REQ_OK or DDT_REQ_BAD_PREFIX    */
 } ddt_attn_args;
 
-/* Bytes of workspace the call will use for these arguments (0 if no split). */
+/* Bytes of workspace the call will use for these arguments (0 if no split).
+ * Reads only the sizes (B, q_len, heads, dims, capacity, max_prefix,
+ * num_splits); pointers may still be unset.  Invalid sizes give 0. */
 DDT_API size_t ddt_verify_attn_workspace_size(const ddt_attn_args* args);
 
-/* Number of KV splits the call will use for these arguments. */
+/* Number of KV splits the call will use for these arguments (same inputs as
+ * ddt_verify_attn_workspace_size; invalid sizes give 1). */
 DDT_API int32_t ddt_verify_attn_num_splits(const ddt_attn_args* args);
 
 DDT_API ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t stream);

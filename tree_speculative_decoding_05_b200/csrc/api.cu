@@ -129,14 +129,21 @@ ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
   return DDT_OK;
 }
 
-static ddt_status check_attn_args(const ddt_attn_args* a) {
+// Sizes and plan parameters only (what the split plan and workspace size need).
+static ddt_status check_attn_shape(const ddt_attn_args* a) {
   if (!a) return DDT_ERR_INVALID_ARG;
   if (a->B < 0 || a->capacity < 0 || a->max_prefix < 0) return DDT_ERR_INVALID_ARG;
   if (a->q_len < 1 || a->q_len > DDT_MAX_Q_LEN || a->num_heads != DDT_NUM_HEADS ||
       a->d_latent != DDT_D_LATENT || a->d_rope != DDT_D_ROPE)
     return DDT_ERR_UNSUPPORTED;
-  if (a->out_dtype != DDT_F32 && a->out_dtype != DDT_BF16) return DDT_ERR_INVALID_ARG;
   if (a->num_splits < 0 || a->num_splits > 64) return DDT_ERR_INVALID_ARG;
+  return DDT_OK;
+}
+
+static ddt_status check_attn_args(const ddt_attn_args* a) {
+  const ddt_status shape = check_attn_shape(a);
+  if (shape != DDT_OK) return shape;
+  if (a->out_dtype != DDT_F32 && a->out_dtype != DDT_BF16) return DDT_ERR_INVALID_ARG;
   if (a->B == 0) return DDT_OK;
   if (!a->prefix_lens || !a->q_lat || !a->q_rope || !a->c_kv || !a->k_rope || !a->mask || !a->out)
     return DDT_ERR_INVALID_ARG;
@@ -152,12 +159,12 @@ static ddt_status check_attn_args(const ddt_attn_args* a) {
 }
 
 int32_t ddt_verify_attn_num_splits(const ddt_attn_args* a) {
-  if (check_attn_args(a) != DDT_OK || a->B == 0) return 1;
+  if (check_attn_shape(a) != DDT_OK || a->B == 0) return 1;
   return verify_num_splits(*a, device_sm_count());
 }
 
 size_t ddt_verify_attn_workspace_size(const ddt_attn_args* a) {
-  if (check_attn_args(a) != DDT_OK || a->B == 0) return 0;
+  if (check_attn_shape(a) != DDT_OK || a->B == 0) return 0;
   return verify_workspace_bytes(*a, verify_num_splits(*a, device_sm_count()));
 }
 
