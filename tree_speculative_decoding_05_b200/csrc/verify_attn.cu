@@ -24,7 +24,9 @@
 //     covering the 512 latent columns (128 TMEM columns each per CTA).  V is the
 //     same c_kv rows read as an MN-major operand (each CTA stages 128 latent
 //     columns x 32 keys = 8 KB per stage).
-//   * TMEM per CTA: S double buffer (2 x 64 cols) + O (256 cols) of 512.
+//   * TMEM per CTA: four S buffers (4 x 64 cols) + O (256 cols) = all 512
+//     columns; four S buffers let S = Q K^T run up to three tiles ahead of the
+//     softmax.
 //   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
 //     half of one query row); warps 4 and 8 TMA producers of the K rings of
 //     even and odd tiles, warp 6 the producer of the V ring; warps 5 and 9
@@ -81,12 +83,15 @@ constexpr int kBarKEmpty = kBarKFull + 2 * kKStages;
 constexpr int kBarVFull = kBarKEmpty + 2 * kKStages;
 constexpr int kBarVEmpty = kBarVFull + kVStages;
 constexpr int kBarQ = kBarVEmpty + kVStages;
-constexpr int kBarS = kBarQ + 1;
-constexpr int kBarP = kBarS + 2;
+constexpr int kBarS = kBarQ + 1;           // four S buffers: S ready
+constexpr int kBarSFree = kBarS + 4;       // four S buffers: read by both CTAs' softmax
+constexpr int kBarP = kBarSFree + 4;
 constexpr int kBarO = kBarP + 2;
 constexpr int kBarQKDone = kBarO + 1;      // two: one per S issuer
 constexpr int kBarPVDone = kBarQKDone + 2;
-constexpr int kNumBars = kBarPVDone + 1;
+constexpr int kBarQFree = kBarPVDone + 1;  // both S issuers are done with this item's Q
+constexpr int kBarOFree = kBarQFree + 1;   // both CTAs' epilogues have read O
+constexpr int kNumBars = kBarOFree + 1;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmemPtr + 4;
 constexpr int kSmemUsed = kOffAbort + 4;
@@ -94,8 +99,9 @@ constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr int kTmemCols = 512;
-constexpr int kTmemS = 0;    // S buffers at columns 0 and 64
-constexpr int kTmemO = 128;  // O halves at columns 128 and 256
+constexpr int kNumS = 4;     // S buffers at columns 0, 64, 128, 192
+constexpr int kTmemS = 0;
+constexpr int kTmemO = 256;  // O halves at columns 256 and 384
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleLog2 = 8.0f;
@@ -123,6 +129,44 @@ __host__ __device__ inline void split_range(int T, int num_splits, int split, in
   t1 = t0 + per < n_tiles ? t0 + per : n_tiles;
 }
 
+// One work item: a pair of tree nodes of one request over one KV split.
+struct WorkItem {
+  int b, pair, split, P, T, t0, ntile, last_tile;
+  bool bad_prefix, valid;
+};
+
+__device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int item) {
+  WorkItem it;
+  const int per_req = p.n_pairs * p.num_splits;
+  it.b = item / per_req;
+  const int rem = item - it.b * per_req;
+  it.pair = rem / p.num_splits;
+  it.split = rem - it.pair * p.num_splits;
+  it.P = p.prefix_lens[it.b];
+  // Requests whose tree block would not fit the cache are rejected as a whole.
+  it.bad_prefix = (it.P < 0) || (static_cast<int64_t>(it.P) + p.Q > p.capacity);
+  it.T = it.P + p.Q;
+  int t0 = 0, t1 = 0;
+  if (!it.bad_prefix) split_range(it.T, p.num_splits, it.split, t0, t1);
+  it.t0 = t0;
+  it.ntile = t1 - t0;  // 0 for an empty split (the merge skips it)
+  it.last_tile = (it.T + 127) / 128 - 1;
+  it.valid = !it.bad_prefix && it.ntile > 0;
+  return it;
+}
+
+// First cache row of KV tile t.  A request's last tile is shifted to end at row
+// T, so no load ever reaches the rows past the tree block (padding that may hold
+// anything); its overlap with the previous tile is masked, and rows below 0
+// (T < 128) read as zeros.
+__device__ __forceinline__ int tile_start(const WorkItem& it, int t) {
+  return t == it.last_tile ? it.T - 128 : 128 * t;
+}
+
+// Persistent kernel: each CTA pair (cluster of 2) loops over work items
+// cluster, cluster + n_clusters, ...  Barriers, rings and tensor memory live
+// across items; per-tile barrier phases follow a tile counter G that counts the
+// tiles of all items a CTA has processed.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     verify_attn_kernel(const __grid_constant__ CUtensorMap tm_qlat,
                        const __grid_constant__ CUtensorMap tm_qrope,
@@ -131,33 +175,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_krope, const VerifyParams p) {
   using namespace va;
   const uint32_t rank = cluster_ctarank();
-  const int item = blockIdx.x >> 1;
-  const int per_req = p.n_pairs * p.num_splits;
-  const int b = item / per_req;
-  const int rem = item - b * per_req;
-  const int pair = rem / p.num_splits;
-  const int split = rem - pair * p.num_splits;
-  const int node = 2 * pair + static_cast<int>(rank);
+  const int cluster = static_cast<int>(blockIdx.x >> 1);
+  const int n_clusters = static_cast<int>(gridDim.x >> 1);
+  const int n_items = p.B * p.n_pairs * p.num_splits;
   const int Q = p.Q;
-  const int P = p.prefix_lens[b];
-
-  // Requests whose tree block would not fit the cache are rejected as a whole;
-  // both CTAs of every pair reach the same decision.
-  const bool bad_prefix = (P < 0) || (static_cast<int64_t>(P) + Q > p.capacity);
-  if (rank == 0 && pair == 0 && split == 0 && threadIdx.x == 0 && p.status)
-    p.status[b] = bad_prefix ? DDT_REQ_BAD_PREFIX : DDT_REQ_OK;
-  if (bad_prefix) return;
-  const int T = P + Q;
-  int t0, t1;
-  split_range(T, p.num_splits, split, t0, t1);
-  if (t0 >= t1) return;  // empty split: the merge skips it
-  const int ntile = t1 - t0;
-  // First cache row of KV tile t.  The request's last tile is shifted to end at
-  // row T, so no load ever reaches the rows past the tree block (padding that
-  // may hold anything); its overlap with the previous tile is masked, and rows
-  // below 0 (T < 128) read as zeros.
-  const int last_tile = (T + 127) / 128 - 1;
-  auto tile_start = [&](int t) -> int { return t == last_tile ? T - 128 : 128 * t; };
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -189,14 +210,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_init(bar(kBarVEmpty + s), 1);
     }
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNumS; ++s) {
       mbar_init(bar(kBarS + s), 1);
-      mbar_init(bar(kBarP + s), 2);  // one arrival per CTA of the pair
+      mbar_init(bar(kBarSFree + s), 2);  // one arrival per CTA of the pair
     }
+    for (int s = 0; s < 2; ++s) mbar_init(bar(kBarP + s), 2);  // one arrival per CTA
     mbar_init(bar(kBarO), 1);
     mbar_init(bar(kBarQKDone + 0), 1);
     mbar_init(bar(kBarQKDone + 1), 1);
     mbar_init(bar(kBarPVDone), 1);
+    mbar_init(bar(kBarQFree), 2);  // a commit of each S issuer
+    mbar_init(bar(kBarOFree), 2);  // one arrival per CTA of the pair
     *abort_flag = 0;
     fence_mbar_init_cluster();
   }
@@ -225,32 +249,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   if (warp == 4 || warp == 8) {
     // ---------------------------------------------- TMA: Q and the K rings
     // Lane 0 issues; warp 4 loads Q and the K stages of even tiles, warp 8 those
-    // of odd tiles.  Only the even CTA arrives on the stage barriers (with the
-    // byte count of both CTAs); both CTAs' loads complete bytes on them.
+    // of odd tiles (by the tile counter G).  Only the even CTA arrives on the
+    // stage barriers (with the byte count of both CTAs); both CTAs' loads
+    // complete bytes on them.
     if (lane == 0) {
       const int g = warp == 4 ? 0 : 1;
       const int key_half = static_cast<int>(rank) * 64;
-      if (g == 0) {
-        const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
-        if (leader) mbar_arrive_expect_tx_local(bar(kBarQ), 2 * kQBytes);
-        for (int c = 0; c < 8; ++c)
-          tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, b);
-        tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, b);
-      }
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
       const uint32_t ring = sKRing + g * kKStages * kStageBytes;
+      const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
       Ring r;
-      for (int jj = g; jj < ntile; jj += 2) {
-        const int key0 = tile_start(t0 + jj) + key_half;
-        for (int c = 0; c < kQChunks; ++c) {
-          mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
-          if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kStageBytes);
-          const uint32_t fb = map_to_rank(bar(full0 + r.stage), 0);
-          const uint32_t dst = ring + r.stage * kStageBytes;
-          if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, b);
-          else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, b);
-          r.advance(kKStages);
+      int iter = 0;
+      int64_t G = 0;
+      for (int item = cluster; item < n_items; item += n_clusters) {
+        const WorkItem it = decode_item(p, item);
+        if (!it.valid) continue;
+        const int node = 2 * it.pair + static_cast<int>(rank);
+        if (g == 0) {
+          // Q of the previous item stays in use until both S issuers are done.
+          if (iter > 0) mbar_wait(bar(kBarQFree), static_cast<uint32_t>((iter - 1) & 1), abort_flag);
+          if (leader) mbar_arrive_expect_tx_local(bar(kBarQ), 2 * kQBytes);
+          for (int c = 0; c < 8; ++c)
+            tma_load_3d_pair(sQ + c * kStageBytes, &tm_qlat, qbar, 64 * c, node * 64, it.b);
+          tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, it.b);
         }
+        for (int jj = 0; jj < it.ntile; ++jj, ++G) {
+          if (static_cast<int>(G & 1) != g) continue;
+          const int key0 = tile_start(it, it.t0 + jj) + key_half;
+          for (int c = 0; c < kQChunks; ++c) {
+            mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
+            if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kStageBytes);
+            const uint32_t fb = map_to_rank(bar(full0 + r.stage), 0);
+            const uint32_t dst = ring + r.stage * kStageBytes;
+            if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, it.b);
+            else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, it.b);
+            r.advance(kKStages);
+          }
+        }
+        ++iter;
       }
     }
     __syncwarp();
@@ -258,18 +294,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     // ------------------------------------------------------------ TMA: V ring
     if (lane == 0) {
       Ring r;
-      for (int jj = 0; jj < ntile; ++jj) {
-        for (int kb = 0; kb < 4; ++kb) {
-          const int key0 = tile_start(t0 + jj) + 32 * kb;
-          for (int nh = 0; nh < 2; ++nh) {
-            mbar_wait(bar(kBarVEmpty + r.stage), r.phase ^ 1u, abort_flag);
-            if (leader) mbar_arrive_expect_tx_local(bar(kBarVFull + r.stage), 2 * kStageBytes);
-            const uint32_t fb = map_to_rank(bar(kBarVFull + r.stage), 0);
-            const int x0 = 256 * nh + 128 * static_cast<int>(rank);
-            const uint32_t dst = sVRing + r.stage * kStageBytes;
-            tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, b);
-            tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, b);
-            r.advance(kVStages);
+      for (int item = cluster; item < n_items; item += n_clusters) {
+        const WorkItem it = decode_item(p, item);
+        if (!it.valid) continue;
+        for (int jj = 0; jj < it.ntile; ++jj) {
+          for (int kb = 0; kb < 4; ++kb) {
+            const int key0 = tile_start(it, it.t0 + jj) + 32 * kb;
+            for (int nh = 0; nh < 2; ++nh) {
+              mbar_wait(bar(kBarVEmpty + r.stage), r.phase ^ 1u, abort_flag);
+              if (leader) mbar_arrive_expect_tx_local(bar(kBarVFull + r.stage), 2 * kStageBytes);
+              const uint32_t fb = map_to_rank(bar(kBarVFull + r.stage), 0);
+              const int x0 = 256 * nh + 128 * static_cast<int>(rank);
+              const uint32_t dst = sVRing + r.stage * kStageBytes;
+              tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, it.b);
+              tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, it.b);
+              r.advance(kVStages);
+            }
           }
         }
       }
@@ -277,32 +317,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     __syncwarp();
   } else if (warp == 5 || warp == 9) {
     // -------------------------------------------------------- MMA: S = Q K^T
-    // Warp 5 issues even tiles into S buffer 0, warp 9 odd tiles into buffer 1.
+    // Warp 5 issues even tiles (by G), warp 9 odd tiles; tile G goes to S
+    // buffer G % 4.
     if (leader && lane == 0) {
       const int g = warp == 5 ? 0 : 1;
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
       const uint32_t ring = sKRing + g * kKStages * kStageBytes;
-      const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(g);
       Ring r;
-      mbar_wait(bar(kBarQ), 0, abort_flag);
-      for (int jj = g; jj < ntile; jj += 2) {
-        if (jj >= 2) {
-          // S buffer g is free once the softmax of tile jj-2 released its P.
-          mbar_wait(bar(kBarP + g), static_cast<uint32_t>(((jj - 2) >> 1) & 1), abort_flag);
-          tc_fence_after_sync();
-        }
-        for (int c = 0; c < kQChunks; ++c) {
-          mbar_wait(bar(full0 + r.stage), r.phase, abort_flag);
-          const uint32_t a0 = sQ + c * kStageBytes;
-          const uint32_t b0 = ring + r.stage * kStageBytes;
+      int iter = 0;
+      int64_t G = 0;
+      for (int item = cluster; item < n_items; item += n_clusters) {
+        const WorkItem it = decode_item(p, item);
+        if (!it.valid) continue;
+        mbar_wait(bar(kBarQ), static_cast<uint32_t>(iter & 1), abort_flag);
+        for (int jj = 0; jj < it.ntile; ++jj, ++G) {
+          if (static_cast<int>(G & 1) != g) continue;
+          const int sbuf = static_cast<int>(G & (kNumS - 1));
+          if (G >= kNumS) {
+            // S buffer sbuf is free once both CTAs' softmax has read tile G-4.
+            mbar_wait(bar(kBarSFree + sbuf), static_cast<uint32_t>(((G >> 2) - 1) & 1), abort_flag);
+            tc_fence_after_sync();
+          }
+          const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(sbuf);
+          for (int c = 0; c < kQChunks; ++c) {
+            mbar_wait(bar(full0 + r.stage), r.phase, abort_flag);
+            const uint32_t a0 = sQ + c * kStageBytes;
+            const uint32_t b0 = ring + r.stage * kStageBytes;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
-                           smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
-          mma_commit<2>(bar(empty0 + r.stage), 0x3);
-          r.advance(kKStages);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
+                             smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
+            mma_commit<2>(bar(empty0 + r.stage), 0x3);
+            r.advance(kKStages);
+          }
+          mma_commit<2>(bar(kBarS + sbuf), 0x3);
         }
-        mma_commit<2>(bar(kBarS + g), 0x3);
+        mma_commit<2>(bar(kBarQFree), 0x3);  // this issuer no longer reads this item's Q
+        ++iter;
       }
       mma_commit<2>(bar(kBarQKDone + g), 0x1);
       mbar_wait(bar(kBarQKDone + g), 0, abort_flag);
@@ -312,26 +363,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     // ------------------------------------------------------- MMA: O += P V
     if (leader && lane == 0) {
       Ring r;
-      for (int jj = 0; jj < ntile; ++jj) {
-        const int pb = jj & 1;
-        mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((jj >> 1) & 1), abort_flag);
-        tc_fence_after_sync();
-        for (int kb = 0; kb < 4; ++kb) {
-          for (int nh = 0; nh < 2; ++nh) {
-            mbar_wait(bar(kBarVFull + r.stage), r.phase, abort_flag);
-            const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
-            const uint32_t a0 = sP + pb * kPBufBytes + (kb >> 1) * kStageBytes + (kb & 1) * 64;
-            const uint32_t b0 = sVRing + r.stage * kStageBytes;
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-              mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
-                             smem_desc_sw128(b0 + 2048 * ks, 4096, 1024), kIdescPV,
-                             !(jj == 0 && kb == 0 && ks == 0));
-            mma_commit<2>(bar(kBarVEmpty + r.stage), 0x3);
-            r.advance(kVStages);
-          }
+      int iter = 0;
+      int64_t G = 0;
+      for (int item = cluster; item < n_items; item += n_clusters) {
+        const WorkItem it = decode_item(p, item);
+        if (!it.valid) continue;
+        if (iter > 0) {
+          // The first P V of an item overwrites O: both CTAs' epilogues must
+          // have read the previous item's O.
+          mbar_wait(bar(kBarOFree), static_cast<uint32_t>((iter - 1) & 1), abort_flag);
+          tc_fence_after_sync();
         }
-        mma_commit<2>(bar(kBarO), 0x3);
+        for (int jj = 0; jj < it.ntile; ++jj, ++G) {
+          const int pb = static_cast<int>(G & 1);
+          mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((G >> 1) & 1), abort_flag);
+          tc_fence_after_sync();
+          for (int kb = 0; kb < 4; ++kb) {
+            for (int nh = 0; nh < 2; ++nh) {
+              mbar_wait(bar(kBarVFull + r.stage), r.phase, abort_flag);
+              const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
+              const uint32_t a0 = sP + pb * kPBufBytes + (kb >> 1) * kStageBytes + (kb & 1) * 64;
+              const uint32_t b0 = sVRing + r.stage * kStageBytes;
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks)
+                mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
+                               smem_desc_sw128(b0 + 2048 * ks, 4096, 1024), kIdescPV,
+                               !(jj == 0 && kb == 0 && ks == 0));
+              mma_commit<2>(bar(kBarVEmpty + r.stage), 0x3);
+              r.advance(kVStages);
+            }
+          }
+          mma_commit<2>(bar(kBarO), 0x3);
+        }
+        ++iter;
       }
       mma_commit<2>(bar(kBarPVDone), 0x1);
       mbar_wait(bar(kBarPVDone), 0, abort_flag);
@@ -343,157 +407,176 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     const int m = t & 63;              // row within this CTA (head)
     const int hf = t >> 6;             // which half of the 128-key tile / O columns
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const bool node_valid = node < Q;
     const int W = (Q + 63) >> 6;
-    uint64_t mw0 = 0, mw1 = 0;
-    if (node_valid) {
-      const uint64_t* mrow = p.mask + (static_cast<int64_t>(b) * Q + node) * W;
-      mw0 = mrow[0];
-      if (W > 1) mw1 = mrow[1];
-    }
     const uint32_t p_full_leader0 = map_to_rank(bar(kBarP), 0);
-    float m_ref = -INFINITY;
-    float l_sum = 0.f;
-    float m_use = 0.f;
-    for (int jj = 0; jj < ntile; ++jj) {
-      const int tile = t0 + jj;
-      const int sb = jj & 1;
-      mbar_wait(bar(kBarS + sb), static_cast<uint32_t>((jj >> 1) & 1), abort_flag);
-      tc_fence_after_sync();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tmem + lane_addr + kTmemS + 64u * sb, r0);
-      tmem_ld32(tmem + lane_addr + kTmemS + 64u * sb + 32u, r1);
-      tmem_wait_ld();
-      float x[64];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(r0[c]) * p.scale_log2;
-        x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
+    const uint32_t s_free_leader0 = map_to_rank(bar(kBarSFree), 0);
+    const uint32_t o_free_leader = map_to_rank(bar(kBarOFree), 0);
+    int64_t G = 0;
+    for (int item = cluster; item < n_items; item += n_clusters) {
+      const WorkItem it = decode_item(p, item);
+      if (rank == 0 && t == 0 && it.pair == 0 && it.split == 0 && p.status)
+        p.status[it.b] = it.bad_prefix ? DDT_REQ_BAD_PREFIX : DDT_REQ_OK;
+      if (!it.valid) continue;
+      const int b = it.b, P = it.P, T = it.T, t0 = it.t0, ntile = it.ntile, split = it.split;
+      const int node = 2 * it.pair + static_cast<int>(rank);
+      const bool node_valid = node < Q;
+      uint64_t mw0 = 0, mw1 = 0;
+      if (node_valid) {
+        const uint64_t* mrow = p.mask + (static_cast<int64_t>(b) * Q + node) * W;
+        mw0 = mrow[0];
+        if (W > 1) mw1 = mrow[1];
       }
-      const int key0 = tile_start(tile) + hf * 64;
-      const int lo = tile * 128;  // keys below lo belong to the previous tile
-      if (key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = key0 + c;
-          bool vis = key < P;
-          if (!vis && key < T) {
-            const int a = key - P;
-            const uint64_t w = a < 64 ? mw0 : mw1;
-            vis = (w >> (a & 63)) & 1ull;
-          }
-          if (key < lo) vis = false;
-          if (!vis) x[c] = -INFINITY;
-        }
-      }
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
-      red_max[sb * 128 + t] = mx;
-      named_barrier_sync(1, kSoftmaxThreads);
-      mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]);
-      float factor = 1.f;
-      bool rescale = false;
-      if (m_ref == -INFINITY) {
-        m_ref = mx;  // nothing accumulated yet: adopt the first finite maximum
-      } else if (mx > m_ref + kRescaleLog2) {
-        factor = fast_exp2(m_ref - mx);
-        m_ref = mx;
-        l_sum *= factor;
-        rescale = true;
-      }
-      m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // The row sum takes the bf16-rounded weights, the values the P V product
-      // multiplies, so the normalised weights sum to one exactly.
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float e0 = fast_exp2(x[2 * c] - m_use);
-        const float e1 = fast_exp2(x[2 * c + 1] - m_use);
-        pk[c] = pack_bf16x2(e0, e1);
-        l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
-      }
-      // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
-      uint8_t* prow = base + kOffP + sb * kPBufBytes + hf * kStageBytes + m * 128;
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
-        uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
-      }
-      if (jj > 0) {
-        // PV of the previous tile must be complete before O may be rescaled.
-        mbar_wait(bar(kBarO), static_cast<uint32_t>((jj - 1) & 1), abort_flag);
+      float m_ref = -INFINITY;
+      float l_sum = 0.f;
+      float m_use = 0.f;
+      for (int jj = 0; jj < ntile; ++jj, ++G) {
+        const int tile = t0 + jj;
+        const int sb = static_cast<int>(G & 1);              // P buffer, exchange slot
+        const int sbuf = static_cast<int>(G & (kNumS - 1));  // S buffer
+        mbar_wait(bar(kBarS + sbuf), static_cast<uint32_t>((G >> 2) & 1), abort_flag);
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int q = 0; q < 8; ++q) {
-            uint32_t o[32];
-            const uint32_t addr = tmem + lane_addr + kTmemO + 32u * q;
-            tmem_ld32(addr, o);
-            tmem_wait_ld();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_addr + kTmemS + 64u * sbuf, r0);
+        tmem_ld32(tmem + lane_addr + kTmemS + 64u * sbuf + 32u, r1);
+        tmem_wait_ld();
+        tc_fence_before_sync();
+        float x[64];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
-            tmem_st32(addr, o);
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(r0[c]) * p.scale_log2;
+          x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
+        }
+        const int key0 = tile_start(it, tile) + hf * 64;
+        const int lo = tile * 128;  // keys below lo belong to the previous tile
+        if (key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int key = key0 + c;
+            bool vis = key < P;
+            if (!vis && key < T) {
+              const int a = key - P;
+              const uint64_t w = a < 64 ? mw0 : mw1;
+              vis = (w >> (a & 63)) & 1ull;
+            }
+            if (key < lo) vis = false;
+            if (!vis) x[c] = -INFINITY;
           }
-          tmem_wait_st();
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+        red_max[sb * 128 + t] = mx;
+        named_barrier_sync(1, kSoftmaxThreads);
+        // Every thread of this CTA has read S: release the buffer.
+        if (t == 0) mbar_arrive_cluster(s_free_leader0 + 8u * sbuf);
+        mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]);
+        float factor = 1.f;
+        bool rescale = false;
+        if (m_ref == -INFINITY) {
+          m_ref = mx;  // nothing accumulated yet: adopt the first finite maximum
+        } else if (mx > m_ref + kRescaleLog2) {
+          factor = fast_exp2(m_ref - mx);
+          m_ref = mx;
+          l_sum *= factor;
+          rescale = true;
+        }
+        m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        // The row sum takes the bf16-rounded weights, the values the P V product
+        // multiplies, so the normalised weights sum to one exactly.
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = fast_exp2(x[2 * c] - m_use);
+          const float e1 = fast_exp2(x[2 * c + 1] - m_use);
+          pk[c] = pack_bf16x2(e0, e1);
+          l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+        }
+        // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
+        uint8_t* prow = base + kOffP + sb * kPBufBytes + hf * kStageBytes + m * 128;
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+          *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
+        }
+        if (jj > 0) {
+          // PV of the previous tile must be complete before O may be rescaled.
+          mbar_wait(bar(kBarO), static_cast<uint32_t>((G - 1) & 1), abort_flag);
+          tc_fence_after_sync();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+            for (int q = 0; q < 8; ++q) {
+              uint32_t o[32];
+              const uint32_t addr = tmem + lane_addr + kTmemO + 32u * q;
+              tmem_ld32(addr, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+              tmem_st32(addr, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        named_barrier_sync(2, kSoftmaxThreads);
+        if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * sb);
+      }
+      // ----------------------------------------------------------- epilogue
+      mbar_wait(bar(kBarO), static_cast<uint32_t>((G - 1) & 1), abort_flag);
+      tc_fence_after_sync();
+      red_l[t] = l_sum;
+      named_barrier_sync(1, kSoftmaxThreads);
+      const float l_row = l_sum + red_l[t ^ 64];
+      const bool empty_row = !(l_row > 0.f);
+      const float inv = empty_row ? 0.f : 1.f / l_row;
+      const float lse_nat = empty_row ? -INFINITY : (m_use + __log2f(l_row)) * kLn2;
+      if (node_valid) {
+        const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
+        const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+#pragma unroll 1
+        for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
+            tmem_wait_ld();
+            const int col = 256 * nh + 128 * hf + 32 * q;
+            if (p.num_splits > 1) {
+              float4* dst = reinterpret_cast<float4*>(
+                  p.part_o + (static_cast<int64_t>(split) * rows_total + row) * 512 + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                     __uint_as_float(o[4 * v + 2]) * inv,
+                                     __uint_as_float(o[4 * v + 3]) * inv);
+            } else if (p.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                     __uint_as_float(o[4 * v + 2]) * inv,
+                                     __uint_as_float(o[4 * v + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * 512 + col);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(
+                    pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                    pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+            }
+          }
+        }
+        if (hf == 0) {
+          if (p.num_splits > 1) p.part_lse[static_cast<int64_t>(split) * rows_total + row] = lse_nat;
+          else if (p.lse) p.lse[row] = lse_nat;
         }
       }
-      fence_proxy_async_smem();
+      // O has been read: the next item's first P V may overwrite it.
       tc_fence_before_sync();
       named_barrier_sync(2, kSoftmaxThreads);
-      if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * sb);
-    }
-    // ------------------------------------------------------------- epilogue
-    mbar_wait(bar(kBarO), static_cast<uint32_t>((ntile - 1) & 1), abort_flag);
-    tc_fence_after_sync();
-    red_l[t] = l_sum;
-    named_barrier_sync(1, kSoftmaxThreads);
-    const float l_row = l_sum + red_l[t ^ 64];
-    const bool empty_row = !(l_row > 0.f);
-    const float inv = empty_row ? 0.f : 1.f / l_row;
-    const float lse_nat = empty_row ? -INFINITY : (m_use + __log2f(l_row)) * kLn2;
-    if (node_valid) {
-      const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
-      const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
-#pragma unroll 1
-      for (int nh = 0; nh < 2; ++nh) {
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
-          tmem_wait_ld();
-          const int col = 256 * nh + 128 * hf + 32 * q;
-          if (p.num_splits > 1) {
-            float4* dst = reinterpret_cast<float4*>(
-                p.part_o + (static_cast<int64_t>(split) * rows_total + row) * 512 + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                   __uint_as_float(o[4 * v + 2]) * inv,
-                                   __uint_as_float(o[4 * v + 3]) * inv);
-          } else if (p.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                   __uint_as_float(o[4 * v + 2]) * inv,
-                                   __uint_as_float(o[4 * v + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * 512 + col);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
-                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
-          }
-        }
-      }
-      if (hf == 0) {
-        if (p.num_splits > 1) p.part_lse[static_cast<int64_t>(split) * rows_total + row] = lse_nat;
-        else if (p.lse) p.lse[row] = lse_nat;
-      }
+      if (t == 0) mbar_arrive_cluster(o_free_leader);
     }
   }
 
@@ -672,8 +755,11 @@ ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* par
   p.n_pairs = (a.q_len + 1) / 2;
   p.out_f32 = a.out_dtype == DDT_F32;
   p.scale_log2 = a.softmax_scale * kLog2e;
-  const int64_t grid = 2ll * a.B * p.n_pairs * num_splits;
-  if (grid > 0x7fffffffll) return DDT_ERR_UNSUPPORTED;
+  // Persistent grid: at most one CTA pair per two SMs; pairs loop over items.
+  const int64_t items = static_cast<int64_t>(a.B) * p.n_pairs * num_splits;
+  if (items > 0x3fffffffll) return DDT_ERR_UNSUPPORTED;
+  const int64_t slots = device_sm_count() / 2 > 0 ? device_sm_count() / 2 : 1;
+  const int64_t grid = 2 * (items < slots ? items : slots);
   verify_attn_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
       m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, p);
   if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
