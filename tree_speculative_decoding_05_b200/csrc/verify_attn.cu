@@ -86,8 +86,8 @@ constexpr int kBarQ = kBarVEmpty + kVStages;
 constexpr int kBarS = kBarQ + 1;           // four S buffers: S ready
 constexpr int kBarSFree = kBarS + 4;       // four S buffers: read by both CTAs' softmax
 constexpr int kBarP = kBarSFree + 4;
-constexpr int kBarO = kBarP + 2;
-constexpr int kBarQKDone = kBarO + 1;      // two: one per S issuer
+constexpr int kBarO = kBarP + 2;           // two: P V of even / odd tiles done
+constexpr int kBarQKDone = kBarO + 2;      // two: one per S issuer
 constexpr int kBarPVDone = kBarQKDone + 2;
 constexpr int kBarQFree = kBarPVDone + 1;  // both S issuers are done with this item's Q
 constexpr int kBarOFree = kBarQFree + 1;   // both CTAs' epilogues have read O
@@ -215,7 +215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_init(bar(kBarSFree + s), 2);  // one arrival per CTA of the pair
     }
     for (int s = 0; s < 2; ++s) mbar_init(bar(kBarP + s), 2);  // one arrival per CTA
-    mbar_init(bar(kBarO), 1);
+    mbar_init(bar(kBarO + 0), 1);
+    mbar_init(bar(kBarO + 1), 1);
     mbar_init(bar(kBarQKDone + 0), 1);
     mbar_init(bar(kBarQKDone + 1), 1);
     mbar_init(bar(kBarPVDone), 1);
@@ -393,7 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
               r.advance(kVStages);
             }
           }
-          mma_commit<2>(bar(kBarO), 0x3);
+          mma_commit<2>(bar(kBarO + static_cast<int>(G & 1)), 0x3);
         }
         ++iter;
       }
@@ -411,6 +412,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     const uint32_t p_full_leader0 = map_to_rank(bar(kBarP), 0);
     const uint32_t s_free_leader0 = map_to_rank(bar(kBarSFree), 0);
     const uint32_t o_free_leader = map_to_rank(bar(kBarOFree), 0);
+    // P V completions are confirmed strictly in tile order (o_next = the next
+    // tile to confirm) on two barriers alternating by tile parity, so a wait
+    // never sees a barrier more than one phase ahead of it.
+    int64_t o_next = 0;
+    auto wait_o_through = [&](int64_t last) {
+      bool waited = false;
+      while (o_next <= last) {
+        mbar_wait(bar(kBarO + static_cast<int>(o_next & 1)), static_cast<uint32_t>((o_next >> 1) & 1),
+                  abort_flag);
+        ++o_next;
+        waited = true;
+      }
+      if (waited) tc_fence_after_sync();
+    };
     int64_t G = 0;
     for (int item = cluster; item < n_items; item += n_clusters) {
       const WorkItem it = decode_item(p, item);
@@ -491,6 +506,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           pk[c] = pack_bf16x2(e0, e1);
           l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
         }
+        // The P buffer of this tile was last read by the P V of tile G-2.
+        wait_o_through(G - 2);
         // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
         uint8_t* prow = base + kOffP + sb * kPBufBytes + hf * kStageBytes + m * 128;
 #pragma unroll
@@ -499,10 +516,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
         }
         if (jj > 0) {
-          // PV of the previous tile must be complete before O may be rescaled.
-          mbar_wait(bar(kBarO), static_cast<uint32_t>((G - 1) & 1), abort_flag);
-          tc_fence_after_sync();
           if (__any_sync(0xffffffffu, rescale)) {
+            // O may be rescaled only once the P V of the previous tile is done
+            // (the next one waits for this tile's P).
+            wait_o_through(G - 1);
 #pragma unroll 1
             for (int q = 0; q < 8; ++q) {
               uint32_t o[32];
@@ -522,8 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * sb);
       }
       // ----------------------------------------------------------- epilogue
-      mbar_wait(bar(kBarO), static_cast<uint32_t>((G - 1) & 1), abort_flag);
-      tc_fence_after_sync();
+      wait_o_through(G - 1);
       red_l[t] = l_sum;
       named_barrier_sync(1, kSoftmaxThreads);
       const float l_row = l_sum + red_l[t ^ 64];
