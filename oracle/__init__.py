@@ -72,6 +72,8 @@ class Oracle:
         lib.oracle_attn_rows.restype = i32
         lib.oracle_tree_accept.argtypes = [P, P, P, P, i32, i32, P, P, P, P]
         lib.oracle_tree_accept.restype = None
+        lib.oracle_tree_build.argtypes = [P, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P]
+        lib.oracle_tree_build.restype = None
         lib.oracle_kv_compact.argtypes = [P, P, i64, i64, i64, i64, i32, i32, i32, P, P, P,
                                           i32, i32, P, P]
         lib.oracle_kv_compact.restype = None
@@ -157,6 +159,27 @@ class Oracle:
                                     _p(bonus), _p(status))
         return path, alen, bonus, status
 
+    def tree_build(self, lp, tok, root_token, q_len):
+        """Best-first draft tree from per-depth top-k log-probs.
+        lp float32 [B,D,K], tok int32 [B,D,K], root_token int32 [B].  Returns a dict of
+        parents, node_tokens, depth (int32 [B,Q]), logw (float32 [B,Q]), next_token,
+        next_sibling (int32 [B,Q]), n_nodes, status (int32 [B])."""
+        lp = _c(lp, np.float32)
+        tok = _c(tok, np.int32)
+        root = _c(root_token, np.int32)
+        B, D, K = lp.shape
+        Q = int(q_len)
+        r = {k: np.zeros((B, Q), dtype=np.int32) for k in ("parents", "node_tokens", "depth",
+                                                           "next_token", "next_sibling")}
+        r["logw"] = np.zeros((B, Q), dtype=np.float32)
+        r["n_nodes"] = np.zeros(B, dtype=np.int32)
+        r["status"] = np.zeros(B, dtype=np.int32)
+        self.lib.oracle_tree_build(_p(lp), _p(tok), _p(root), B, D, K, Q, _p(r["parents"]),
+                                   _p(r["node_tokens"]), _p(r["depth"]), _p(r["logw"]),
+                                   _p(r["next_token"]), _p(r["next_sibling"]), _p(r["n_nodes"]),
+                                   _p(r["status"]))
+        return r
+
     def kv_compact(self, c_kv, k_rope, prefix_lens, path, accept_len, capacity=None):
         """Compaction on copies of the caches (uint16 [B,cap,DL] / [B,cap,DR]).
         Returns (c_kv', k_rope', new_prefix_lens, status)."""
@@ -212,3 +235,7 @@ def tree_accept(*args, **kwargs):
 
 def kv_compact(*args, **kwargs):
     return default().kv_compact(*args, **kwargs)
+
+
+def tree_build(*args, **kwargs):
+    return default().tree_build(*args, **kwargs)

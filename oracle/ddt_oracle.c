@@ -307,3 +307,112 @@ void oracle_kv_compact(uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs, int64_t
     if (new_prefix_lens) new_prefix_lens[b] = P + alen;
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Tree build.  [Foundation] "The Single-Threaded Heap Design" (best-first     */
+/* expansion of a draft tree from per-depth top-k log-probabilities, budget   */
+/* and depth bounded), "Tie-Breaking and Numerical Precision" (equal weights  */
+/* are taken in insertion order; float32 arithmetic), "Assumptions Underlying */
+/* the Design" (4: the sibling weight is the parent-relative expression       */
+/* logw - lp[depth-1][rank] + lp[depth-1][rank+1], in that order; 5: with     */
+/* topk = 1 the candidates can run out before the budget).                    */
+/*                                                                            */
+/* Per request: lp[d][r], tok[d][r] for d < D, r < K (row d describes tree    */
+/* depth d+1), and the root's token.  Node 0 is the root: depth 0, logw 0,    */
+/* parent -1.  A candidate is (logw, depth d, rank r, parent).  The first     */
+/* candidate is (0 + lp[0][0], 1, 0, 0).  While fewer than Q nodes exist and  */
+/* a candidate remains: take the candidate of largest logw (among equals the  */
+/* one inserted first); it becomes the next node n with that parent, depth,   */
+/* logw and token tok[d-1][r].  Then insert, first                            */
+/*   its first child  (logw + lp[d][0], d+1, 0, n)                 if d < D,  */
+/* then                                                                       */
+/*   its next sibling ((logw - lp[d-1][r]) + lp[d-1][r+1], d, r+1, parent)   */
+/*                                                                 if r+1 < K.*/
+/* logw arithmetic is binary32 with round-to-nearest, in the order shown.     */
+/*                                                                            */
+/* Retrieve pointers: next_token[i] = smallest child index of i, next_sibling */
+/* [i] = next larger node index with the same parent (-1 where none).         */
+/* Slots n_nodes <= i < Q (when candidates ran out) are padding: parent 0,    */
+/* token -1, depth 1, logw -inf, linked into no list.  Every lp entry must be */
+/* finite, else status BAD_LP and the tree is the root alone plus padding.    */
+/* The candidate list is kept in insertion order (removal shifts the rest),   */
+/* so the first maximum found by a scan is the earliest inserted one.         */
+/* ------------------------------------------------------------------------ */
+enum { ORC_BAD_LP = 6 };
+
+typedef struct {
+  float logw;
+  int depth, rank, parent;
+} orc_candidate;
+
+void oracle_tree_build(const float* lp, const int32_t* tok, const int32_t* root_token, int B,
+                       int D, int K, int Q, int32_t* parents, int32_t* node_tokens,
+                       int32_t* depth, float* logw, int32_t* next_token, int32_t* next_sibling,
+                       int32_t* n_nodes, int32_t* status) {
+  orc_candidate* cand = (orc_candidate*)malloc(sizeof(orc_candidate) * (size_t)(2 * Q + 2));
+  for (int b = 0; b < B; ++b) {
+    const float* L = lp + (size_t)b * D * K;
+    const int32_t* T = tok + (size_t)b * D * K;
+    int32_t* par = parents + (size_t)b * Q;
+    int32_t* ntk = node_tokens + (size_t)b * Q;
+    int32_t* dep = depth + (size_t)b * Q;
+    float* lw = logw + (size_t)b * Q;
+    int32_t* first = next_token + (size_t)b * Q;
+    int32_t* sib = next_sibling + (size_t)b * Q;
+    int st = ORC_OK;
+    for (int e = 0; e < D * K; ++e)
+      if (!isfinite(L[e])) st = ORC_BAD_LP;
+
+    par[0] = -1;
+    ntk[0] = root_token[b];
+    dep[0] = 0;
+    lw[0] = 0.0f;
+    int n = 1, ncand = 0;
+    if (st == ORC_OK && Q > 1) {
+      float root_w = 0.0f;
+      cand[ncand++] = (orc_candidate){root_w + L[0], 1, 0, 0};
+    }
+    while (n < Q && ncand > 0) {
+      int best = 0;
+      for (int c = 1; c < ncand; ++c)
+        if (cand[c].logw > cand[best].logw) best = c;
+      orc_candidate x = cand[best];
+      memmove(cand + best, cand + best + 1, sizeof(orc_candidate) * (size_t)(ncand - best - 1));
+      ncand -= 1;
+      const int node = n++;
+      par[node] = x.parent;
+      ntk[node] = T[(size_t)(x.depth - 1) * K + x.rank];
+      dep[node] = x.depth;
+      lw[node] = x.logw;
+      if (x.depth < D) {
+        float w = x.logw + L[(size_t)x.depth * K + 0];
+        cand[ncand++] = (orc_candidate){w, x.depth + 1, 0, node};
+      }
+      if (x.rank + 1 < K) {
+        float w = x.logw - L[(size_t)(x.depth - 1) * K + x.rank];
+        w = w + L[(size_t)(x.depth - 1) * K + x.rank + 1];
+        cand[ncand++] = (orc_candidate){w, x.depth, x.rank + 1, x.parent};
+      }
+    }
+    for (int i = n; i < Q; ++i) {
+      par[i] = 0;
+      ntk[i] = -1;
+      dep[i] = 1;
+      lw[i] = -INFINITY;
+    }
+    for (int i = 0; i < Q; ++i) first[i] = sib[i] = -1;
+    for (int i = 1; i < n; ++i) { /* children in ascending index */
+      int p = par[i];
+      if (first[p] == -1) {
+        first[p] = i;
+      } else {
+        int c = first[p];
+        while (sib[c] != -1) c = sib[c];
+        sib[c] = i;
+      }
+    }
+    if (n_nodes) n_nodes[b] = n;
+    if (status) status[b] = st;
+  }
+  free(cand);
+}

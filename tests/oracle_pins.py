@@ -321,9 +321,127 @@ def pin_compact_golden(orc):
         assert np.array_equal(kr2[0], np.array(case["k_rope"], np.uint16)), case["name"]
 
 
+# ---------------------------------------------------------------------------
+# Tree build
+# ---------------------------------------------------------------------------
+
+def _num(v):
+    return float(v)  # JSON holds "nan" / "-inf" as strings; float() reads both
+
+
+def pin_build_golden(orc):
+    """Hand-traced expansions ([Foundation] "The Single-Threaded Heap Design",
+    "Tie-Breaking and Numerical Precision", "Assumptions Underlying the Design")."""
+    for case in _golden("tree_build_cases.json")["cases"]:
+        lp = np.array([[[_num(x) for x in row] for row in case["lp"]]], dtype=np.float32)
+        r = orc.tree_build(lp, np.array([case["tok"]], np.int32),
+                           np.array([case["root_token"]], np.int32), case["q_len"])
+        for k in ("parents", "node_tokens", "depth", "next_token", "next_sibling"):
+            assert r[k][0].tolist() == case[k], (case["name"], k)
+        want = np.array([_num(x) for x in case["logw"]], dtype=np.float32)
+        assert np.array_equal(r["logw"][0], want), case["name"]
+        assert r["n_nodes"][0] == case["n_nodes"] and r["status"][0] == case["status"], case["name"]
+
+
+def _int_lp(seed, D, K, lo=1, hi=4000):
+    """Log-probs that are negative integers / 16 (exact in float32 and in every
+    partial sum used here), sorted descending per depth."""
+    s = inputs.stream_base(seed, 90, 0)
+    mags = (lo + inputs.raw_u64(s, 0, D * K) % np.uint64(hi - lo)).astype(np.int64).reshape(D, K)
+    mags.sort(axis=1)
+    return -mags, (-mags).astype(np.float32) / 16.0
+
+
+def pin_build_bruteforce(orc):
+    """With every row of lp non-positive and sorted descending, a node never
+    outweighs its parent or its previous sibling, so best-first expansion creates
+    nodes in globally descending weight: the tree is the Q-1 heaviest nodes of
+    the full K-ary tree of depth D.  Enumerate that full tree with exact integer
+    weights and compare node set, creation order, parents, tokens, depth, logw."""
+    import itertools
+    checked = 0
+    for seed in range(40):
+        D, K, Q = 3 + seed % 2, 3, 12 + seed % 9
+        ilp, lp = _int_lp(seed, D, K)
+        tok = (1000 * np.arange(1, D + 1)[:, None] + np.arange(K)[None, :]).astype(np.int32)
+        nodes = []  # (exact weight, rank path)
+        for d in range(1, D + 1):
+            for ranks in itertools.product(range(K), repeat=d):
+                nodes.append((sum(int(ilp[k, r]) for k, r in enumerate(ranks)), ranks))
+        nodes.sort(key=lambda x: -x[0])
+        top = nodes[:Q - 1]
+        weights = [w for w, _ in nodes[:Q]]
+        if len(set(weights)) < len(weights):
+            continue  # a tie at or inside the cut: the order is not fixed by weights alone
+        checked += 1
+        r = orc.tree_build(lp[None], tok[None], np.array([7], np.int32), Q)
+        index = {(): 0}
+        for n, (w, ranks) in enumerate(top, start=1):
+            index[ranks] = n
+            assert r["parents"][0, n] == index[ranks[:-1]]
+            assert r["depth"][0, n] == len(ranks)
+            assert r["node_tokens"][0, n] == tok[len(ranks) - 1, ranks[-1]]
+            assert r["logw"][0, n] == np.float32(w / 16.0)
+        assert r["n_nodes"][0] == Q and r["status"][0] == 0
+    assert checked >= 20
+
+
+def pin_build_closed_forms(orc):
+    """topk = 1 gives a chain of min(D, Q-1) drafts; depth 1 gives a star of
+    min(K, Q-1) children of the root in rank order."""
+    for D, Q in ((5, 9), (9, 5), (1, 2)):
+        lp = -np.arange(1, D + 1, dtype=np.float32)[:, None] / 4
+        tok = np.arange(D, dtype=np.int32)[:, None] + 100
+        r = orc.tree_build(lp[None], tok[None], np.array([3], np.int32), Q)
+        n = 1 + min(D, Q - 1)
+        assert r["n_nodes"][0] == n
+        assert r["parents"][0, :n].tolist() == list(range(-1, n - 1))
+        assert r["node_tokens"][0, 1:n].tolist() == list(range(100, 100 + n - 1))
+        cum = np.cumsum(np.arange(1, n)) / 4  # exact quarters
+        assert np.array_equal(r["logw"][0, 1:n], (-cum).astype(np.float32))
+        assert (r["node_tokens"][0, n:] == -1).all() and (r["parents"][0, n:] == 0).all()
+    for K, Q in ((6, 4), (3, 8)):
+        lp = -np.arange(1, K + 1, dtype=np.float32)[None, :] / 8
+        tok = np.arange(K, dtype=np.int32)[None, :] + 50
+        r = orc.tree_build(lp[None], tok[None], np.array([3], np.int32), Q)
+        n = 1 + min(K, Q - 1)
+        assert r["n_nodes"][0] == n
+        assert (r["parents"][0, 1:n] == 0).all()
+        assert r["node_tokens"][0, 1:n].tolist() == list(range(50, 50 + n - 1))
+        assert np.array_equal(r["logw"][0, 1:n], lp[0, :n - 1])
+        assert r["next_token"][0, 0] == 1
+        assert r["next_sibling"][0, 1:n].tolist() == list(range(2, n)) + [-1]
+
+
+def pin_build_structure(orc):
+    """On random float log-probs (any order): parents precede children, depth is the
+    parent's plus one and at most D, each node's token is a token of its depth row,
+    and next_token / next_sibling list each node's children in ascending index."""
+    B, D, K, Q = 24, 6, 5, 33
+    s = inputs.stream_base(5, 91, 0)
+    lp = (inputs.normal(s, B * D * K) * 2.0).astype(np.float32).reshape(B, D, K)
+    tok = np.arange(B * D * K, dtype=np.int32).reshape(B, D, K)
+    r = orc.tree_build(lp, tok, np.arange(B, dtype=np.int32), Q)
+    assert (r["status"] == 0).all() and (r["n_nodes"] == Q).all()
+    for b in range(B):
+        par, dep = r["parents"][b], r["depth"][b]
+        assert par[0] == -1 and dep[0] == 0
+        for i in range(1, Q):
+            assert 0 <= par[i] < i and dep[i] == dep[par[i]] + 1 <= D
+            assert r["node_tokens"][b, i] in tok[b, dep[i] - 1]
+        for i in range(Q):
+            kids = [c for c in range(1, Q) if par[c] == i]
+            walk, c = [], r["next_token"][b, i]
+            while c != -1:
+                walk.append(int(c))
+                c = r["next_sibling"][b, c]
+            assert walk == kids
+
+
 ALL_PINS = [
     pin_mask_golden, pin_mask_bruteforce, pin_mask_closed_forms,
     pin_attn_chain_is_causal, pin_attn_decode, pin_attn_tiny_bruteforce, pin_attn_probs,
     pin_attn_prefix_permutation, pin_attn_zero_query, pin_attn_single_key,
     pin_attn_duplicate_keys, pin_accept_golden, pin_accept_properties, pin_compact_golden,
+    pin_build_golden, pin_build_bruteforce, pin_build_closed_forms, pin_build_structure,
 ]

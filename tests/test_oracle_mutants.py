@@ -25,6 +25,17 @@ MUTANTS = [
      "memcpy(ckv + (int64_t)(P + i + (i + 1 < alen)) * ckv_rs"),
     ("depth off by one", "depth[i] = (i == 0) ? 0 : depth[parents[i]] + 1;",
      "depth[i] = (i == 0) ? 1 : depth[parents[i]] + 1;"),
+    ("sibling weight keeps the node's own log-prob",
+     "float w = x.logw - L[(size_t)(x.depth - 1) * K + x.rank];", "float w = x.logw;"),
+    ("child weight from the node's own depth row", "float w = x.logw + L[(size_t)x.depth * K + 0];",
+     "float w = x.logw + L[(size_t)(x.depth - 1) * K + 0];"),
+    ("ties go to the latest insertion", "if (cand[c].logw > cand[best].logw) best = c;",
+     "if (cand[c].logw >= cand[best].logw) best = c;"),
+    ("token from rank 0", "ntk[node] = T[(size_t)(x.depth - 1) * K + x.rank];",
+     "ntk[node] = T[(size_t)(x.depth - 1) * K];"),
+    ("sibling hangs under the node", "cand[ncand++] = (orc_candidate){w, x.depth, x.rank + 1, x.parent};",
+     "cand[ncand++] = (orc_candidate){w, x.depth, x.rank + 1, node};"),
+    ("children stop one level early", "if (x.depth < D) {", "if (x.depth + 1 < D) {"),
 ]
 
 
