@@ -63,8 +63,14 @@ namespace va {
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kStageBytes = 8192;
-constexpr int kKStages = 4;                        // each of the two K rings (even / odd tiles)
-constexpr int kVStages = 6;                        // V ring (feeds O += P V)
+#ifndef DDT_VERIFY_K_STAGES
+#define DDT_VERIFY_K_STAGES 4
+#endif
+#ifndef DDT_VERIFY_V_STAGES
+#define DDT_VERIFY_V_STAGES 6
+#endif
+constexpr int kKStages = DDT_VERIFY_K_STAGES;      // each of the two K rings (even / odd tiles)
+constexpr int kVStages = DDT_VERIFY_V_STAGES;      // V ring (feeds O += P V)
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
 constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
@@ -74,7 +80,10 @@ constexpr int kOffVRing = kOffKRing + 2 * kKStages * kStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffRedMax = kOffP + 2 * kPBufBytes;     // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
-constexpr int kOffBar = kOffRedL + 128 * 4;
+constexpr int kMaxSortedB = 512;  // requests ordered by length (larger B: natural order)
+constexpr int kOffLen = kOffRedL + 128 * 4;            // int32[kMaxSortedB]
+constexpr int kOffOrder = kOffLen + kMaxSortedB * 4;   // int32[kMaxSortedB]
+constexpr int kOffBar = kOffOrder + kMaxSortedB * 4;
 // barriers: two K rings' full/empty (ring g at offset g * kKStages), V ring
 // full/empty, q_full, s_full[2], p_full[2], o_done, and one "all issued MMAs
 // done" barrier per issuing thread (two S issuers, one O issuer).
@@ -135,11 +144,14 @@ struct WorkItem {
   bool bad_prefix, valid;
 };
 
-__device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int item) {
+// Work index w -> item.  With `order` (requests sorted by decreasing cache
+// length) the w-th item belongs to request order[w / per_req].
+__device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int w, const int* order) {
   WorkItem it;
   const int per_req = p.n_pairs * p.num_splits;
-  it.b = item / per_req;
-  const int rem = item - it.b * per_req;
+  const int slot = w / per_req;
+  it.b = order ? order[slot] : slot;
+  const int rem = w - slot * per_req;
   it.pair = rem / p.num_splits;
   it.split = rem - it.pair * p.num_splits;
   it.P = p.prefix_lens[it.b];
@@ -163,10 +175,19 @@ __device__ __forceinline__ int tile_start(const WorkItem& it, int t) {
   return t == it.last_tile ? it.T - 128 : 128 * t;
 }
 
-// Persistent kernel: each CTA pair (cluster of 2) loops over work items
-// cluster, cluster + n_clusters, ...  Barriers, rings and tensor memory live
-// across items; per-tile barrier phases follow a tile counter G that counts the
-// tiles of all items a CTA has processed.
+// The k-th work index of a cluster: rounds of n_clusters indices, alternating
+// direction ("snake"), so that with items sorted by decreasing cost each pair
+// gets a balanced mix (a static longest-first schedule).  -1 past the end.
+__device__ __forceinline__ int work_index(int k, int cluster, int n_clusters, int n_items) {
+  const int64_t w = static_cast<int64_t>(k) * n_clusters +
+                    ((k & 1) ? (n_clusters - 1 - cluster) : cluster);
+  return w < n_items ? static_cast<int>(w) : -1;
+}
+
+// Persistent kernel: each CTA pair (cluster of 2) loops over the work indices
+// work_index(0, ...), work_index(1, ...), ...  Barriers, rings and tensor memory
+// live across items; per-tile barrier phases follow a tile counter G that
+// counts the tiles of all items a CTA has processed.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     verify_attn_kernel(const __grid_constant__ CUtensorMap tm_qlat,
                        const __grid_constant__ CUtensorMap tm_qrope,
@@ -178,6 +199,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   const int cluster = static_cast<int>(blockIdx.x >> 1);
   const int n_clusters = static_cast<int>(gridDim.x >> 1);
   const int n_items = p.B * p.n_pairs * p.num_splits;
+  const int n_rounds = (n_items + n_clusters - 1) / n_clusters;
   const int Q = p.Q;
 
   extern __shared__ uint8_t smem_raw[];
@@ -229,10 +251,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     tmem_alloc<2>(smem_u32(tmem_ptr_smem), kTmemCols);
     tmem_relinquish<2>();
   }
+  // Requests ranked by decreasing cache length (ties by index), computed
+  // redundantly by every CTA from prefix_lens: one warp per request counts, over
+  // its lanes, the requests that come before it.  Invalid prefixes rank as empty.
+  int* len_smem = reinterpret_cast<int*>(base + kOffLen);
+  int* order_smem = reinterpret_cast<int*>(base + kOffOrder);
+  const bool sorted = p.B <= kMaxSortedB;
+  if (sorted) {
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+      const int P = p.prefix_lens[b];
+      len_smem[b] = (P < 0 || static_cast<int64_t>(P) + Q > p.capacity) ? 0 : P + Q;
+    }
+    __syncthreads();
+    for (int bi = warp; bi < p.B; bi += kThreads / 32) {
+      const int li = len_smem[bi];
+      int before = 0;
+      for (int bj = lane; bj < p.B; bj += 32) {
+        const int lj = len_smem[bj];
+        before += (lj > li) || (lj == li && bj < bi);
+      }
+      before = __reduce_add_sync(0xffffffffu, before);
+      if (lane == 0) order_smem[before] = bi;
+    }
+  }
   tc_fence_before_sync();
   cluster_sync();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_ptr_smem;
+  const int* order = sorted ? order_smem : nullptr;
 
   // Ring helper: a stage index and phase bit advancing over `n` stages.
   struct Ring {
@@ -262,8 +308,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       Ring r;
       int iter = 0;
       int64_t G = 0;
-      for (int item = cluster; item < n_items; item += n_clusters) {
-        const WorkItem it = decode_item(p, item);
+      for (int k = 0; k < n_rounds; ++k) {
+        const int item = work_index(k, cluster, n_clusters, n_items);
+        if (item < 0) continue;
+        const WorkItem it = decode_item(p, item, order);
         if (!it.valid) continue;
         const int node = 2 * it.pair + static_cast<int>(rank);
         if (g == 0) {
@@ -295,8 +343,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     // ------------------------------------------------------------ TMA: V ring
     if (lane == 0) {
       Ring r;
-      for (int item = cluster; item < n_items; item += n_clusters) {
-        const WorkItem it = decode_item(p, item);
+      for (int k = 0; k < n_rounds; ++k) {
+        const int item = work_index(k, cluster, n_clusters, n_items);
+        if (item < 0) continue;
+        const WorkItem it = decode_item(p, item, order);
         if (!it.valid) continue;
         for (int jj = 0; jj < it.ntile; ++jj) {
           for (int kb = 0; kb < 4; ++kb) {
@@ -327,8 +377,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       Ring r;
       int iter = 0;
       int64_t G = 0;
-      for (int item = cluster; item < n_items; item += n_clusters) {
-        const WorkItem it = decode_item(p, item);
+      for (int k = 0; k < n_rounds; ++k) {
+        const int item = work_index(k, cluster, n_clusters, n_items);
+        if (item < 0) continue;
+        const WorkItem it = decode_item(p, item, order);
         if (!it.valid) continue;
         mbar_wait(bar(kBarQ), static_cast<uint32_t>(iter & 1), abort_flag);
         for (int jj = 0; jj < it.ntile; ++jj, ++G) {
@@ -366,8 +418,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       Ring r;
       int iter = 0;
       int64_t G = 0;
-      for (int item = cluster; item < n_items; item += n_clusters) {
-        const WorkItem it = decode_item(p, item);
+      for (int k = 0; k < n_rounds; ++k) {
+        const int item = work_index(k, cluster, n_clusters, n_items);
+        if (item < 0) continue;
+        const WorkItem it = decode_item(p, item, order);
         if (!it.valid) continue;
         if (iter > 0) {
           // The first P V of an item overwrites O: both CTAs' epilogues must
@@ -427,8 +481,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       if (waited) tc_fence_after_sync();
     };
     int64_t G = 0;
-    for (int item = cluster; item < n_items; item += n_clusters) {
-      const WorkItem it = decode_item(p, item);
+    for (int k = 0; k < n_rounds; ++k) {
+      const int item = work_index(k, cluster, n_clusters, n_items);
+      if (item < 0) continue;
+      const WorkItem it = decode_item(p, item, order);
       if (rank == 0 && t == 0 && it.pair == 0 && it.split == 0 && p.status)
         p.status[it.b] = it.bad_prefix ? DDT_REQ_BAD_PREFIX : DDT_REQ_OK;
       if (!it.valid) continue;
