@@ -25,6 +25,7 @@ there is no collective on the data path, only the timing reduction.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import json
 import math
@@ -40,6 +41,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+from tree_speculative_decoding_05_b200 import inputs  # noqa: E402  (seeded generator only)
 
 METRIC = "verify-attn µs/call & TFLOP/s (% bf16 peak), 64 streams × q_len 33 × 4K prefix"
 H, DL, DR = 64, 512, 64
@@ -317,6 +320,258 @@ def run_reference(args, w):
 # Main (GPU arm)
 # ---------------------------------------------------------------------------
 
+DRAFT_DEPTH, DRAFT_TOPK = 15, 8  # drafter rows (tree depth <= 15) and candidates per row
+
+
+def graph_time_us(fn, n: int, flush=None, reps: int = 5) -> float:
+    """Mean device time of one fn() call: n calls back to back captured in one CUDA
+    graph (so host launch overhead is not timed), the graph replayed `reps` times
+    with events around each replay, median of those.  With `flush` (a buffer larger
+    than L2), every call is preceded by a write of it, and a graph of the n writes
+    alone is timed the same way and subtracted."""
+    import torch
+
+    def capture(body):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            body()  # untimed warm-up outside the capture
+            side.synchronize()
+            with torch.cuda.graph(g, stream=side):
+                for k in range(n):
+                    body(k)
+        torch.cuda.current_stream().wait_stream(side)
+        return g
+
+    def replay_ms(g):
+        g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return statistics.median(times)
+
+    def with_flush(k=0):
+        if flush is not None:
+            flush.fill_(k & 0xFF)
+        fn()
+
+    total = replay_ms(capture(with_flush))
+    if flush is not None:
+        total -= replay_ms(capture(lambda k=0: flush.fill_(k & 0xFF)))
+    return max(total, 0.0) / n * 1e3
+
+
+def time_extras(w, d, host, mask, out, lse, workspace, max_prefix, stream, flush, iters,
+                warmup):
+    """Mean device time (us) of the calls outside the benchmark step, each timed as
+    `iters` calls in one CUDA graph (L2 flushed before every call when the inputs
+    fit in it, the flush's own time subtracted):
+    the tree build of drafts of the workload's shape; tree_accept then kv_compact
+    against the fused accept_compact; and one chained decode step (tree build, block
+    write, verify, accept + compaction) replayed from a CUDA graph with its state
+    reset by the graph itself."""
+    import torch
+
+    from tree_speculative_decoding_05_b200 import ddt
+
+    dev = d["q_lat"].device
+    B, Q = w.B, w.q_len
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        return graph_time_us(fn, iters, flush)
+
+    draft = inputs.draft_batch(w.seed, B, DRAFT_DEPTH, DRAFT_TOPK)
+    lp = torch.from_numpy(draft.lp).to(dev)
+    tok = torch.from_numpy(draft.tok).to(dev)
+    root = torch.from_numpy(draft.root_token).to(dev)
+    tb = ddt.tree_build(lp, tok, root, Q)
+    res = {"draft": f"{DRAFT_DEPTH} rows x top-{DRAFT_TOPK} per request"}
+    res["tree_build_us"] = timed(lambda: ddt.tree_build(lp, tok, root, Q, out=tb))
+
+    i32 = lambda shape: torch.empty(shape, dtype=torch.int32, device=dev)
+    path, alen, bonus, ast, newp, cst = i32((B, Q)), i32(B), i32(B), i32(B), i32(B), i32(B)
+
+    def separate():
+        ddt.tree_accept(d["node_tokens"], d["target_tokens"], d["next_token"], d["next_sibling"],
+                        path=path, accept_len=alen, bonus=bonus, status=ast)
+        ddt.kv_compact(d["c_kv"], d["k_rope"], d["prefix"], path, alen, new_prefix_lens=newp,
+                       status=cst)
+
+    def fused():
+        ddt.accept_compact(d["node_tokens"], d["target_tokens"], d["next_token"],
+                           d["next_sibling"], d["c_kv"], d["k_rope"], d["prefix"], path=path,
+                           accept_len=alen, bonus=bonus, accept_status=ast,
+                           new_prefix_lens=newp, compact_status=cst)
+
+    res["accept_then_compact_us"] = timed(separate)
+    res["accept_compact_us"] = timed(fused)
+
+    # Chained decode step: the workload's queries and its own tree-block rows,
+    # drafts as above, and a target continuation that follows the drafter's top
+    # token with probability 0.7.
+    rows = torch.from_numpy(np.stack([np.arange(int(p), int(p) + Q) for p in w.prefix_lens]))
+    bidx = torch.arange(B)[:, None]
+    u = inputs.uniform(inputs.stream_base(w.seed, 97, 0), 0, B * Q).reshape(B, Q)
+    cont = np.where((u < 0.7) & (np.arange(Q)[None, :] < DRAFT_DEPTH),
+                    draft.tok[:, np.minimum(np.arange(Q), DRAFT_DEPTH - 1), 0], 31999)
+    step = dict(lp=lp, tok=tok, q_lat=d["q_lat"], q_rope=d["q_rope"],
+                block_ckv=host["c_kv"][bidx, rows].contiguous().to(dev),
+                block_krope=host["k_rope"][bidx, rows].contiguous().to(dev),
+                target_continuation=torch.from_numpy(cont.astype(np.int32)).to(dev))
+    state = dict(c_kv=d["c_kv"], k_rope=d["k_rope"], prefix_lens=d["prefix"].clone(),
+                 root_token=root.clone())
+    p0, r0 = d["prefix"].clone(), root.clone()
+    bufs = dict(mask=mask, out=out, lse=lse, workspace=workspace, verify_status=i32(B),
+                parents=i32((B, Q)), node_tokens=i32((B, Q)), depth=i32((B, Q)),
+                next_token=i32((B, Q)), next_sibling=i32((B, Q)), n_nodes=i32(B),
+                target_tokens=i32((B, Q)), path=path, accept_len=alen, status=i32((4, B)))
+    dargs = ddt.decode_step_args(state, step, bufs, w.softmax_scale, max_prefix)
+
+    def one_step():
+        state["prefix_lens"].copy_(p0)
+        state["root_token"].copy_(r0)
+        ddt.decode_step(dargs)
+
+    one_step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            one_step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    for k, (a, b) in enumerate(evs):
+        if flush is not None:
+            flush.fill_(k & 0xFF)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    res["decode_step_us"] = sum(a.elapsed_time(b) for a, b in evs) / iters * 1e3
+    st = bufs["status"].cpu().numpy()
+    res["decode_step_statuses_ok"] = bool((st == 0).all() and
+                                          (bufs["verify_status"].cpu().numpy() == 0).all())
+    res["decode_step_mean_accept_len"] = float(alen.float().mean().item())
+    res["decode_step_kernels"] = 4 + (1 if workspace is not None else 0)
+    del graph
+    return res
+
+
+def per_call_report(args) -> int:
+    """Every call of the path timed alone per workload: 10 warm-up calls, then 100
+    calls captured back to back in a CUDA graph and the replay timed with events,
+    median of 5 replays; with a warm L2, and with a 256 MB write before every call
+    (the writes' own time subtracted).  The oracle runs on the same workload (configs
+    0 and 1 whole; larger ones on a sample of query rows) with all host threads and
+    with one."""
+    import torch
+
+    import oracle
+    from tree_speculative_decoding_05_b200 import ddt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = measured_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
+
+    def timed(fn, flushed):
+        # 10 untimed calls, then 100 calls per graph, median of 5 replays
+        for _ in range(10):
+            fn()
+        return graph_time_us(fn, 100, flush if flushed else None, reps=5)
+
+    for cfg in [int(c) for c in args.configs.split(",") if c.strip()]:
+        w = inputs.config(cfg)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+        q_lat, q_rope, c_kv, k_rope = bf(w.q_lat), bf(w.q_rope), bf(w.c_kv), bf(w.k_rope)
+        prefix, parents = i32(w.prefix_lens), i32(w.parents)
+        nt, tt, fc, ns = (i32(w.node_tokens), i32(w.target_tokens), i32(w.next_token),
+                          i32(w.next_sibling))
+        B, Q = w.B, w.q_len
+        max_prefix = int(w.prefix_lens.max())
+        mask, depth, mst = ddt.build_mask(parents)
+        od = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+        out = torch.empty((B, Q, H, DL), dtype=od, device=dev)
+        lse = torch.empty((B, Q, H), dtype=torch.float32, device=dev) if w.want_lse else None
+        ws, splits = ddt.verify_attn_workspace_size(q_lat, q_rope, c_kv, k_rope, prefix, mask,
+                                                    w.softmax_scale, max_prefix)
+        wsp = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev) if ws else None
+        a_st = ddt._attn_args(q_lat, q_rope, c_kv, k_rope, prefix, mask, w.softmax_scale, out,
+                              lse, max_prefix, 0, None, None)
+        ws_st = int(ddt.load().ddt_verify_attn_split_tail_workspace_size(ctypes.byref(a_st)))
+        wsp_st = torch.empty(ws_st, dtype=torch.uint8, device=dev)
+        path, alen = torch.empty((B, Q), dtype=torch.int32, device=dev), \
+            torch.empty((B,), dtype=torch.int32, device=dev)
+        ddt.tree_accept(nt, tt, fc, ns, path=path, accept_len=alen)
+        newp = torch.empty((B,), dtype=torch.int32, device=dev)
+        draft = inputs.draft_batch(w.seed, B, DRAFT_DEPTH, DRAFT_TOPK)
+        lp, tok, root = (torch.from_numpy(draft.lp).to(dev), torch.from_numpy(draft.tok).to(dev),
+                         torch.from_numpy(draft.root_token).to(dev))
+        tb = ddt.tree_build(lp, tok, root, Q)
+        calls = {
+            "tree_build": lambda: ddt.tree_build(lp, tok, root, Q, out=tb),
+            "build_mask": lambda: ddt.build_mask(parents, mask=mask, depth=depth, status=mst),
+            "verify_attn": lambda: ddt.verify_attn(q_lat, q_rope, c_kv, k_rope, prefix, mask,
+                                                   w.softmax_scale, max_prefix=max_prefix,
+                                                   out=out, lse=lse, workspace=wsp),
+            "verify_attn_split_tail": lambda: ddt.verify_attn(
+                q_lat, q_rope, c_kv, k_rope, prefix, mask, w.softmax_scale,
+                max_prefix=max_prefix, out=out, lse=lse, workspace=wsp_st, split_tail=True),
+            "tree_accept": lambda: ddt.tree_accept(nt, tt, fc, ns, path=path, accept_len=alen),
+            "kv_compact": lambda: ddt.kv_compact(c_kv, k_rope, prefix, path, alen,
+                                                 new_prefix_lens=newp),
+            "accept_compact": lambda: ddt.accept_compact(nt, tt, fc, ns, c_kv, k_rope, prefix,
+                                                         path=path, accept_len=alen,
+                                                         new_prefix_lens=newp),
+        }
+        res = {}
+        for name, fn in calls.items():
+            res[name] = {"warm_us": timed(fn, False), "l2_flushed_us": timed(fn, True)}
+        flops = verify_flops(w.prefix_lens, w.parents)
+        for name in ("verify_attn", "verify_attn_split_tail"):
+            us = res[name]["l2_flushed_us"]
+            res[name]["tflops"] = flops / (us * 1e-6) / 1e12
+            res[name]["frac_of_peak"] = res[name]["tflops"] / peak
+        # the oracle: whole workload for the two small configs, else a row sample
+        total = B * Q * H
+        rng = np.random.RandomState(cfg)
+        rows = np.arange(total, dtype=np.int64) if cfg in (0, 1) else \
+            np.sort(rng.choice(total, size=min(total, 4096), replace=False)).astype(np.int64)
+        orc = {}
+        for label, nth in (("all_threads", 0), ("one_thread", 1)):
+            if nth == 1 and cfg not in (0, 1):
+                continue
+            t0 = time.perf_counter()
+            oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens, w.parents,
+                             w.softmax_scale, rows, nthreads=nth)
+            secs = time.perf_counter() - t0
+            orc[label] = {"seconds": secs, "rows": int(len(rows)),
+                          "tflops": flops_rows(w.prefix_lens, w.parents, rows) / secs / 1e12}
+        orc["threads"] = oracle.threads()
+        print(json.dumps({"workload": w.name, "config": cfg, "kv_splits": splits,
+                          "peak_tflops": peak, "peak_source": f"{peak_src} burst bf16",
+                          "calls_us": res, "oracle": orc}), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -327,13 +582,27 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--per-call", action="store_true",
+                    help="instead of the step benchmark: every call of the path timed alone on "
+                         "each workload (10 warm-up + 100 timed calls, median of 5 repetitions, "
+                         "warm L2 and after a 256 MB L2 flush), plus the oracle on all host "
+                         "cores and on one; one JSON line per workload")
+    ap.add_argument("--configs", type=str, default="0,1,2,3,4")
+    ap.add_argument("--shard", choices=["replicas", "lpt"], default="replicas",
+                    help="with several GPUs: every rank runs its own batch of the workload "
+                         "(replicas, weak scaling) or the ranks split one batch by request "
+                         "with the longest-first rule (strong scaling)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the timings of the calls outside the step (tree build, fused "
+                         "accept+compaction, chained decode step)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     world, rank, local = dist_env()
-    from tree_speculative_decoding_05_b200 import inputs
 
+    if args.per_call:
+        return per_call_report(args)
     if args.impl == "reference":
         if rank != 0:
             return 0
@@ -347,8 +616,15 @@ def main(argv=None) -> int:
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
-    # Every rank runs its own batch of the same shape (independent requests).
+    # Every rank runs its own batch of the same shape (independent requests), or,
+    # with --shard lpt, its longest-first share of one batch.
     w = inputs.config(args.config)
+    if args.shard == "lpt" and world > 1:
+        from tree_speculative_decoding_05_b200.sharding import lpt_partition, request_costs
+        part = lpt_partition(request_costs(w.prefix_lens, w.q_len), world)[rank]
+        if len(part) == 0:
+            raise SystemExit("--shard lpt: more ranks than requests")
+        w = inputs.subset(w, part)
 
     def bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
@@ -507,6 +783,12 @@ def main(argv=None) -> int:
                            "the tree block's KV rows and the tree arrays are copied in and "
                            "the accepted tokens read back"}
 
+    # ---- calls outside the step: tree build, fused accept+compaction, decode step
+    extras = None
+    if not args.no_extras:
+        extras = time_extras(w, d, host, mask, out, lse, workspace if ws_bytes else None,
+                             max_prefix, stream, flush, max(args.steps, 20), args.warmup)
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -532,13 +814,15 @@ def main(argv=None) -> int:
             "warmup": args.warmup,
             "ms_per_step": step_ms_max,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if (args.shard == "lpt" and world > 1) else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": w.name, "B": B, "q_len": Q, "heads": H,
                        "prefix": max_prefix, "out": w.out_dtype, "kv_splits": splits,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "parallelism": ("single GPU" if world == 1 else
+                                       f"requests split longest-first over {world} GPUs"
+                                       if args.shard == "lpt" else f"replicas x{world}"),
                        "l2": ("inputs %.0f MB per GPU, over twice the L2: no flush" % (
                                   input_bytes / 1e6)) if flush is None else
                              ("inputs %.0f MB per GPU: L2 flushed (256 MB write) between "
@@ -553,6 +837,7 @@ def main(argv=None) -> int:
                          "traffic": measured_traffic(args.config),
                          "algorithmic_bytes": bytes_local,
                          "kernel": "verify_attn_kernel"},
+            "extras": extras,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,

@@ -1,13 +1,17 @@
 /*
  * ddt.h — C ABI of the DDTree tree-verify library for NVIDIA B200 (sm_100a).
  *
- * Four calls make up the verification step of draft-tree speculative decoding
- * on a multi-head-latent-attention (MLA) model:
+ * The calls below build a draft tree and verify it, one step of draft-tree
+ * speculative decoding on a multi-head-latent-attention (MLA) model:
  *
+ *   ddt_tree_build   best-first draft tree from per-depth top-k log-probabilities
  *   ddt_build_mask   per-node ancestor-or-self visibility bitmask from parents[]
  *   ddt_verify_attn  tree-verify MLA-absorb attention over the latent KV cache
  *   ddt_tree_accept  greedy longest-match walk of the draft tree
  *   ddt_kv_compact   gather of the accepted rows into the contiguous prefix
+ *   ddt_accept_compact  the last two in one launch
+ *   ddt_kv_write_block  the tree block's KV rows into the cache after the prefix
+ *   ddt_decode_step  all of the above chained on the device for one decode step
  *
  * Sources (cited by page title and section):
  *   [Race Conditions]  "Race Conditions, Buffer Aliasing, and the Architecture of
@@ -72,6 +76,7 @@ typedef enum ddt_status {
 #define DDT_REQ_WALK_LIMIT 3   /* the tree walk examined more than q_len nodes     */
 #define DDT_REQ_BAD_PREFIX 4   /* prefix_len < 0 or prefix_len + rows > capacity   */
 #define DDT_REQ_BAD_LENGTH 5   /* accept_len not in [1, q_len]                     */
+#define DDT_REQ_BAD_LP 6       /* a log-probability given to the tree build is not finite */
 
 typedef enum ddt_dtype { DDT_F32 = 0, DDT_BF16 = 1 } ddt_dtype;
 
@@ -82,6 +87,55 @@ typedef enum ddt_dtype { DDT_F32 = 0, DDT_BF16 = 1 } ddt_dtype;
 
 /* Mask words per node for a given q_len. */
 #define DDT_MASK_WORDS(q_len) (((q_len) + 63) / 64)
+
+/* ------------------------------------------------------------------------ */
+/* ddt_tree_build                                                           */
+/* ------------------------------------------------------------------------ */
+/* Best-first construction of the draft tree of each request.
+ *
+ * Source: [Foundation] "The Single-Threaded Heap Design" (one serial best-first
+ * expansion per request; budget <= 64 and depth <= 15 fit on chip; the other
+ * threads build the visibility matrix and the retrieve pointers), "Tie-Breaking
+ * and Numerical Precision" (equal weights in insertion order; float32), and
+ * "Assumptions Underlying the Design" (item 4: the sibling weight expression;
+ * item 5: candidates can run out before the budget, e.g. with topk = 1).
+ *
+ * Inputs per request b: lp[b,d,r] and tok[b,d,r] for d < D (depth_levels),
+ * r < K (topk): the drafter's log-probabilities and tokens at tree depth d+1,
+ * best first (the build does not require the order, but only with rows sorted
+ * descending is it a best-first search); root_token[b].
+ *
+ * Expansion (the reading adopted where the pages are silent: a picked node
+ * inserts its first child before its next sibling):
+ *   node 0 = root: parent -1, depth 0, logw 0, token root_token[b]
+ *   candidates = [(0 + lp[0,0], depth 1, rank 0, parent 0)]
+ *   while nodes < q_len and candidates remain:
+ *     take the candidate of largest logw (the earliest inserted among equals)
+ *     -> node n: parent, depth d, logw, token tok[d-1, r]
+ *     if d < D:     insert (logw + lp[d,0], d+1, 0, n)
+ *     if r+1 < K:   insert ((logw - lp[d-1,r]) + lp[d-1,r+1], d, r+1, parent)
+ *   All logw arithmetic is float32, rounded to nearest, in exactly this order.
+ *
+ * Outputs, int32 [B, q_len] unless noted:
+ *   parents, node_tokens; depth (or NULL); logw float [B, q_len] (or NULL);
+ *   next_token[i] = smallest child index of i, next_sibling[i] = the next larger
+ *   index with the same parent (-1 where none) — the retrieve pointers that
+ *   ddt_tree_accept walks; mask uint64 [B, q_len, W] (or NULL) as ddt_build_mask
+ *   would compute it from parents; n_nodes int32 [B] (or NULL); status int32
+ *   [B] (or NULL).
+ * Node slots n_nodes <= i < q_len (candidates ran out) are padding: parent 0,
+ * token -1, depth 1, logw -inf, visibility {0, i}, in no child list, so no walk
+ * reaches them.  A non-finite lp entry sets DDT_REQ_BAD_LP and leaves the root
+ * alone (n_nodes = 1) with padding.
+ * Errors: B < 0, depth_levels < 1, topk < 1 -> DDT_ERR_INVALID_ARG; q_len
+ * outside [1,128] -> DDT_ERR_UNSUPPORTED; lp, tok, root_token, parents,
+ * node_tokens, next_token or next_sibling NULL with B > 0 -> DDT_ERR_INVALID_ARG.
+ * B = 0 is a no-op. */
+DDT_API ddt_status ddt_tree_build(const float* lp, const int32_t* tok, const int32_t* root_token,
+                          int32_t B, int32_t depth_levels, int32_t topk, int32_t q_len,
+                          int32_t* parents, int32_t* node_tokens, int32_t* depth, float* logw,
+                          int32_t* next_token, int32_t* next_sibling, uint64_t* mask,
+                          int32_t* n_nodes, int32_t* status, ddt_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* ddt_build_mask                                                           */
@@ -207,6 +261,27 @@ DDT_API ddt_status ddt_verify_attn_noalloc(const ddt_attn_args* args, ddt_stream
 DDT_API size_t ddt_verify_attn_noalloc_scratch_bytes(void);
 
 /* ------------------------------------------------------------------------ */
+/* ddt_verify_attn_split_tail                                               */
+/* ------------------------------------------------------------------------ */
+/* The same attention as ddt_verify_attn, computed the way the pages planned
+ * their production engine: a dense pass over the prefix rows [0, P) (every
+ * node sees all of them; split across SMs like the split-KV plan), a small pass
+ * over the tree block [P, P+q_len) with the visibility mask, and an LSE merge of
+ * the partials:  lse = ln(e^lse_prefix + e^lse_tree),
+ * out = e^(lse_prefix - lse) out_prefix + e^(lse_tree - lse) out_tree.
+ * Source: [Foundation] "Assumptions Underlying the Design" (item 2: a library
+ * kernel for the long prefix, the custom kernel only for the small tree tail)
+ * and [Verdict] "The Timeout That Tells a Story".  It exists to measure that
+ * design against the single fused pass of ddt_verify_attn; results agree with
+ * it within the attention tolerance (the summation order differs).
+ * Arguments as for ddt_verify_attn, except that the workspace is required:
+ * at least ddt_verify_attn_split_tail_workspace_size(args) bytes, 256-byte
+ * aligned, else DDT_ERR_INVALID_ARG and nothing is launched.  num_splits, when
+ * positive, forces the number of prefix splits. */
+DDT_API size_t ddt_verify_attn_split_tail_workspace_size(const ddt_attn_args* args);
+DDT_API ddt_status ddt_verify_attn_split_tail(const ddt_attn_args* args, ddt_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* ddt_tree_accept                                                          */
 /* ------------------------------------------------------------------------ */
 /* Greedy acceptance of the longest draft path that the target agrees with.
@@ -257,7 +332,8 @@ DDT_API ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* ta
  * c_kv / k_rope: bf16 caches with the strides of ddt_verify_attn (elements,
  * multiples of 8, 16-byte aligned bases); rows are 512 / 64 values.
  * path int32 [B, q_len] (entries read for i < accept_len only), accept_len
- * int32 [B], prefix_lens int32 [B], new_prefix_lens int32 [B] or NULL.
+ * int32 [B], prefix_lens int32 [B], new_prefix_lens int32 [B] or NULL (it may
+ * be prefix_lens itself, updated in place).
  * status int32 [B] or NULL: DDT_REQ_BAD_LENGTH, DDT_REQ_BAD_INDEX (a path entry
  * outside [0, q_len)) or DDT_REQ_BAD_PREFIX (P < 0 or P + q_len > capacity);
  * a request with a non-zero status is left unchanged and its new prefix equals
@@ -269,6 +345,110 @@ DDT_API ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_st
                           const int32_t* accept_len, int32_t B, int32_t q_len,
                           int32_t* new_prefix_lens, int32_t* status,
                           ddt_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* ddt_accept_compact                                                       */
+/* ------------------------------------------------------------------------ */
+/* ddt_tree_accept followed by ddt_kv_compact of its path, in one launch.
+ *
+ * Source: [Race Conditions] "Race Conditions, Buffer Aliasing, and the
+ * Architecture of a Native DDTree Inference Engine" (the compaction gather of
+ * the accepted rows; fusing that gather is named there as work still to do)
+ * and the walk of ddt_tree_accept.  Results are exactly those of the two calls
+ * in sequence: path, accept_len, bonus_token and accept_status as
+ * ddt_tree_accept writes them, then the cache rows, new_prefix_lens and
+ * compact_status as ddt_kv_compact writes them for that path (which can only
+ * report DDT_REQ_BAD_PREFIX, since the walk's path is always in range).
+ * new_prefix_lens may be prefix_lens itself (updated in place); bonus_token,
+ * accept_status, new_prefix_lens and compact_status may be NULL.  Arguments and
+ * errors as for the two calls. */
+DDT_API ddt_status ddt_accept_compact(const int32_t* node_tokens, const int32_t* target_tokens,
+                              const int32_t* next_token, const int32_t* next_sibling,
+                              int32_t B, int32_t q_len, void* c_kv, void* k_rope,
+                              int64_t ckv_batch_stride, int64_t ckv_row_stride,
+                              int64_t kr_batch_stride, int64_t kr_row_stride, int32_t capacity,
+                              const int32_t* prefix_lens, int32_t* path, int32_t* accept_len,
+                              int32_t* bonus_token, int32_t* accept_status,
+                              int32_t* new_prefix_lens, int32_t* compact_status,
+                              ddt_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* ddt_kv_write_block                                                       */
+/* ------------------------------------------------------------------------ */
+/* Writes the tree block's KV rows into the cache right after the prefix.
+ *
+ * Source: [Race Conditions] "The Cache Compaction Problem" (the tree's KV goes
+ * into the cache at the offset of the prefix; node i is row P+i).
+ *
+ *   for i < q_len:  c_kv row P+i <- block_ckv[b,i,:],  k_rope row P+i <- block_krope[b,i,:]
+ *
+ * block_ckv bf16 [B, q_len, 512] and block_krope bf16 [B, q_len, 64], both
+ * contiguous and 16-byte aligned; caches and strides as for ddt_verify_attn.
+ * status int32 [B] or NULL: DDT_REQ_BAD_PREFIX (P < 0 or P + q_len > capacity,
+ * nothing written for that request).  Errors as for ddt_kv_compact. */
+DDT_API ddt_status ddt_kv_write_block(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
+                              int64_t ckv_row_stride, int64_t kr_batch_stride,
+                              int64_t kr_row_stride, int32_t capacity,
+                              const int32_t* prefix_lens, const void* block_ckv,
+                              const void* block_krope, int32_t B, int32_t q_len,
+                              int32_t* status, ddt_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* ddt_decode_step                                                          */
+/* ------------------------------------------------------------------------ */
+/* One speculative decode step chained on the device, for every request:
+ *   1. ddt_tree_build   from this step's draft (lp, tok) and root_token
+ *   2. ddt_kv_write_block of this step's tree-block rows at the prefix, and the
+ *      target's greedy token after each node, target_tokens[b,i] =
+ *      target_continuation[b, depth[b,i]]
+ *   3. ddt_verify_attn  with the tree's mask
+ *   4. ddt_accept_compact, writing the bonus token into root_token and the new
+ *      prefix length into attn.prefix_lens (both are the state of the next step)
+ * Source: [Race Conditions] "The Mission: A Native DDTree Engine" and "The Cache
+ * Compaction Problem" (build, verify, accept, compact, in that order, with the
+ * tree block written at the prefix offset), [Verdict] "What Was Learned"
+ * (chaining the tree builder's output into the accept walk).
+ *
+ * The model's own work (the drafter, the target model's KV rows, queries and
+ * greedy tokens) is outside this library: its results arrive as inputs — lp and
+ * tok [B, D, K], the tree block's KV rows, the absorbed queries (attn.q_lat,
+ * attn.q_rope), and target_continuation int32 [B, q_len], where entry d is the
+ * target's greedy token after the accepted path of depth d.  Under greedy
+ * verification that token does not depend on which path of that depth was
+ * taken once the path matches the target, so a per-depth continuation gives
+ * every node on a matching path its exact target token.
+ *
+ * The call only launches kernels (four, or five with split-KV), in order, on
+ * `stream`; it neither allocates nor synchronises, so it can be captured in a
+ * CUDA graph.  attn.max_prefix sizes the split-KV plan (any prefix is handled;
+ * a bound near the real prefixes plans best).  The step writes through
+ * attn.mask (the tree's visibility words), attn.c_kv / attn.k_rope (the tree
+ * block, then the compaction), attn.prefix_lens (the new prefix) and
+ * attn.status (the verify status).
+ * status int32 [4, B] or NULL: rows = tree build, block write, accept,
+ * compaction.  Every output array is caller-owned and [B, q_len] unless noted. */
+typedef struct ddt_decode_args {
+  ddt_attn_args attn;                 /* verify; prefix_lens is updated in place */
+  int32_t depth_levels, topk;         /* D, K of the draft */
+  const float* lp;                    /* [B, D, K] */
+  const int32_t* tok;                 /* [B, D, K] */
+  int32_t* root_token;                /* [B]: this step's root; the bonus token after */
+  const void* block_ckv;              /* bf16 [B, q_len, 512] */
+  const void* block_krope;            /* bf16 [B, q_len, 64] */
+  const int32_t* target_continuation; /* [B, q_len] */
+  int32_t* parents;
+  int32_t* node_tokens;
+  int32_t* depth;
+  int32_t* next_token;
+  int32_t* next_sibling;
+  int32_t* n_nodes;                   /* [B] or NULL */
+  int32_t* target_tokens;
+  int32_t* path;
+  int32_t* accept_len;                /* [B] */
+  int32_t* status;                    /* [4, B] or NULL */
+} ddt_decode_args;
+
+DDT_API ddt_status ddt_decode_step(const ddt_decode_args* args, ddt_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 DDT_API const char* ddt_status_str(ddt_status status);

@@ -26,9 +26,10 @@ def declared_functions():
     return sorted(set(re.findall(r"DDT_API\s+[\w\s\*]+?\b(ddt_\w+)\s*\(", text)))
 
 
-def test_header_declares_the_four_calls():
+def test_header_declares_the_path_calls():
     names = declared_functions()
-    for n in ("ddt_build_mask", "ddt_verify_attn", "ddt_tree_accept", "ddt_kv_compact"):
+    for n in ("ddt_build_mask", "ddt_verify_attn", "ddt_tree_accept", "ddt_kv_compact",
+              "ddt_tree_build", "ddt_accept_compact", "ddt_kv_write_block", "ddt_decode_step"):
         assert n in names
 
 
@@ -41,19 +42,21 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, n)
 
 
-def test_attn_args_layout_matches_c(tmp_path):
+@pytest.mark.parametrize("cname,pystruct", [("ddt_attn_args", ddt.AttnArgs),
+                                             ("ddt_decode_args", ddt.DecodeArgs)])
+def test_args_struct_layout_matches_c(tmp_path, cname, pystruct):
     src = tmp_path / "layout.c"
-    fields = [f for f, _ in ddt.AttnArgs._fields_]
-    body = "\n".join(f'  printf("{f} %zu\\n", offsetof(ddt_attn_args, {f}));' for f in fields)
+    fields = [f for f, _ in pystruct._fields_]
+    body = "\n".join(f'  printf("{f} %zu\\n", offsetof({cname}, {f}));' for f in fields)
     src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "ddt.h"\nint main(void){\n'
-                   f'  printf("sizeof %zu\\n", sizeof(ddt_attn_args));\n{body}\n  return 0;\n}}\n')
+                   f'  printf("sizeof %zu\\n", sizeof({cname}));\n{body}\n  return 0;\n}}\n')
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o",
                            str(exe)])
     got = dict(line.split() for line in subprocess.check_output([str(exe)], text=True).splitlines())
-    assert int(got["sizeof"]) == ctypes.sizeof(ddt.AttnArgs)
+    assert int(got["sizeof"]) == ctypes.sizeof(pystruct)
     for f in fields:
-        assert int(got[f]) == getattr(ddt.AttnArgs, f).offset, f
+        assert int(got[f]) == getattr(pystruct, f).offset, f
 
 
 def test_host_argument_checks(lib):
@@ -82,6 +85,31 @@ def test_host_argument_checks(lib):
     assert lib.ddt_verify_attn(ctypes.byref(a), None) == ddt.DDT_ERR_INVALID_ARG
     a.B = 0
     assert lib.ddt_verify_attn(ctypes.byref(a), None) == ddt.DDT_OK
+    # tree build: sizes, then null pointers; B = 0 is a no-op
+    tb = lambda B, D, K, Q, p=None: lib.ddt_tree_build(p, p, p, B, D, K, Q, p, p, None, None, p, p,
+                                                        None, None, None, None)
+    assert tb(1, 15, 8, 129) == ddt.DDT_ERR_UNSUPPORTED
+    assert tb(1, 15, 8, 0) == ddt.DDT_ERR_UNSUPPORTED
+    assert tb(1, 0, 8, 33) == ddt.DDT_ERR_INVALID_ARG
+    assert tb(1, 15, 0, 33) == ddt.DDT_ERR_INVALID_ARG
+    assert tb(-1, 15, 8, 33) == ddt.DDT_ERR_INVALID_ARG
+    assert tb(2, 15, 8, 33) == ddt.DDT_ERR_INVALID_ARG
+    assert tb(0, 15, 8, 33) == ddt.DDT_OK
+    assert lib.ddt_accept_compact(None, None, None, None, 1, 129, None, None, 0, 512, 0, 64, 300,
+                                  None, None, None, None, None, None, None,
+                                  None) == ddt.DDT_ERR_UNSUPPORTED
+    assert lib.ddt_accept_compact(None, None, None, None, 1, 9, None, None, 0, 512, 0, 64, 300,
+                                  None, None, None, None, None, None, None,
+                                  None) == ddt.DDT_ERR_INVALID_ARG
+    assert lib.ddt_kv_write_block(None, None, 0, 512, 0, 64, 300, None, None, None, 1, 9, None,
+                                  None) == ddt.DDT_ERR_INVALID_ARG
+    assert lib.ddt_kv_write_block(None, None, 0, 512, 0, 64, 300, None, None, None, 0, 9, None,
+                                  None) == ddt.DDT_OK
+    d = ddt.DecodeArgs()
+    d.attn = ddt.AttnArgs(B=1, q_len=9, num_heads=64, d_latent=512, d_rope=64, capacity=300)
+    d.depth_levels, d.topk = 15, 8
+    assert lib.ddt_decode_step(ctypes.byref(d), None) == ddt.DDT_ERR_INVALID_ARG
+    assert lib.ddt_decode_step(None, None) == ddt.DDT_ERR_INVALID_ARG
     assert lib.ddt_status_str(ddt.DDT_ERR_CUDA) == b"CUDA error"
     assert b"sm_100a" in lib.ddt_version()
 

@@ -67,3 +67,49 @@ def test_work_accounting_matches_definition():
     assert f == 64 * 2 * 1088 * vis
     rows = np.arange(2 * 5 * 64)
     assert bench.flops_rows(prefix, parents, rows) == pytest.approx(f)
+
+
+def _shard_worker(rank: int, world: int, port: int, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch
+    import torch.distributed as dist
+
+    import bench
+    from tree_speculative_decoding_05_b200 import inputs
+    from tree_speculative_decoding_05_b200.sharding import lpt_partition, request_costs
+
+    bench.init_dist(world, "gloo")
+    try:
+        P = inputs.ragged_prefixes(1003, 64, 256, 8192)  # the ragged workload's prefixes
+        mine = lpt_partition(request_costs(P, 65), world)[rank]
+        counts = [torch.zeros(1, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(counts, torch.tensor([len(mine)]))
+        n_max = int(max(c.item() for c in counts))
+        padded = torch.full((n_max,), -1, dtype=torch.int64)
+        padded[:len(mine)] = torch.from_numpy(mine)
+        got = [torch.empty(n_max, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(got, padded)
+        load = float(request_costs(P, 65)[mine].sum())
+        q.put((rank, sorted(int(x) for g in got for x in g.tolist() if x >= 0), load))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_requests_split_longest_first_over_two_ranks():
+    """Each rank derives the same longest-first partition and takes its part: the
+    parts cover every request exactly once and their loads are balanced."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for _, union, _ in results:
+        assert union == list(range(64))
+    loads = [r[2] for r in results]
+    assert abs(loads[0] - loads[1]) <= 8192 + 65

@@ -92,6 +92,23 @@ ddt_status ddt_build_mask(const int32_t* parents, int32_t B, int32_t q_len, uint
   return DDT_OK;
 }
 
+ddt_status ddt_tree_build(const float* lp, const int32_t* tok, const int32_t* root_token,
+                          int32_t B, int32_t depth_levels, int32_t topk, int32_t q_len,
+                          int32_t* parents, int32_t* node_tokens, int32_t* depth, float* logw,
+                          int32_t* next_token, int32_t* next_sibling, uint64_t* mask,
+                          int32_t* n_nodes, int32_t* status, ddt_stream_t stream) {
+  if (B < 0 || depth_levels < 1 || topk < 1) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!lp || !tok || !root_token || !parents || !node_tokens || !next_token || !next_sibling)
+    return DDT_ERR_INVALID_ARG;
+  if (launch_tree_build(lp, tok, root_token, B, depth_levels, topk, q_len, parents, node_tokens,
+                        depth, logw, next_token, next_sibling, mask, n_nodes, status,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
 ddt_status ddt_tree_accept(const int32_t* node_tokens, const int32_t* target_tokens,
                            const int32_t* next_token, const int32_t* next_sibling, int32_t B,
                            int32_t q_len, int32_t* path, int32_t* accept_len,
@@ -125,6 +142,35 @@ ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
                         ckv_batch_stride, ckv_row_stride, kr_batch_stride, kr_row_stride, capacity,
                         prefix_lens, path, accept_len, B, q_len, new_prefix_lens, status,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
+ddt_status ddt_accept_compact(const int32_t* node_tokens, const int32_t* target_tokens,
+                              const int32_t* next_token, const int32_t* next_sibling, int32_t B,
+                              int32_t q_len, void* c_kv, void* k_rope, int64_t ckv_batch_stride,
+                              int64_t ckv_row_stride, int64_t kr_batch_stride,
+                              int64_t kr_row_stride, int32_t capacity,
+                              const int32_t* prefix_lens, int32_t* path, int32_t* accept_len,
+                              int32_t* bonus_token, int32_t* accept_status,
+                              int32_t* new_prefix_lens, int32_t* compact_status,
+                              ddt_stream_t stream) {
+  if (B < 0 || capacity < 0) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!node_tokens || !target_tokens || !next_token || !next_sibling || !c_kv || !k_rope ||
+      !prefix_lens || !path || !accept_len)
+    return DDT_ERR_INVALID_ARG;
+  if (!aligned16(c_kv) || !aligned16(k_rope)) return DDT_ERR_INVALID_ARG;
+  if (!cache_strides_ok(B, capacity, ckv_batch_stride, ckv_row_stride, kr_batch_stride,
+                        kr_row_stride))
+    return DDT_ERR_INVALID_ARG;
+  if (launch_accept_compact(node_tokens, target_tokens, next_token, next_sibling, B, q_len,
+                            static_cast<uint16_t*>(c_kv), static_cast<uint16_t*>(k_rope),
+                            ckv_batch_stride, ckv_row_stride, kr_batch_stride, kr_row_stride,
+                            capacity, prefix_lens, path, accept_len, bonus_token, accept_status,
+                            new_prefix_lens, compact_status,
+                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DDT_ERR_CUDA;
   return DDT_OK;
 }
@@ -185,6 +231,90 @@ ddt_status ddt_verify_attn(const ddt_attn_args* a, ddt_stream_t stream) {
     }
   }
   return launch_verify_attn(*a, splits, part_o, part_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ddt_verify_attn_split_tail_workspace_size(const ddt_attn_args* a) {
+  if (check_attn_shape(a) != DDT_OK || a->B == 0) return 0;
+  return verify_workspace_bytes(*a, verify_num_splits(*a, device_sm_count()) + 1);
+}
+
+ddt_status ddt_verify_attn_split_tail(const ddt_attn_args* a, ddt_stream_t stream) {
+  const ddt_status st = check_attn_args(a);
+  if (st != DDT_OK || a->B == 0) return st;
+  const int splits = verify_num_splits(*a, device_sm_count());
+  const size_t need = verify_workspace_bytes(*a, splits + 1);
+  if (!a->workspace || a->workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return DDT_ERR_INVALID_ARG;
+  float* part_o = static_cast<float*>(a->workspace);
+  float* part_lse = part_o + static_cast<size_t>(splits + 1) * a->B * a->q_len * 64 * 512;
+  return launch_verify_attn_split_tail(*a, splits, part_o, part_lse,
+                                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+ddt_status ddt_kv_write_block(void* c_kv, void* k_rope, int64_t ckv_batch_stride,
+                              int64_t ckv_row_stride, int64_t kr_batch_stride,
+                              int64_t kr_row_stride, int32_t capacity,
+                              const int32_t* prefix_lens, const void* block_ckv,
+                              const void* block_krope, int32_t B, int32_t q_len,
+                              int32_t* status, ddt_stream_t stream) {
+  if (B < 0 || capacity < 0) return DDT_ERR_INVALID_ARG;
+  if (q_len < 1 || q_len > DDT_MAX_Q_LEN) return DDT_ERR_UNSUPPORTED;
+  if (B == 0) return DDT_OK;
+  if (!c_kv || !k_rope || !prefix_lens || !block_ckv || !block_krope) return DDT_ERR_INVALID_ARG;
+  if (!aligned16(c_kv) || !aligned16(k_rope) || !aligned16(block_ckv) || !aligned16(block_krope))
+    return DDT_ERR_INVALID_ARG;
+  if (!cache_strides_ok(B, capacity, ckv_batch_stride, ckv_row_stride, kr_batch_stride,
+                        kr_row_stride))
+    return DDT_ERR_INVALID_ARG;
+  if (launch_kv_write_block(static_cast<uint16_t*>(c_kv), static_cast<uint16_t*>(k_rope),
+                            ckv_batch_stride, ckv_row_stride, kr_batch_stride, kr_row_stride,
+                            capacity, prefix_lens, static_cast<const uint16_t*>(block_ckv),
+                            static_cast<const uint16_t*>(block_krope), B, q_len, nullptr, nullptr,
+                            nullptr, status, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
+}
+
+ddt_status ddt_decode_step(const ddt_decode_args* d, ddt_stream_t stream) {
+  if (!d) return DDT_ERR_INVALID_ARG;
+  const ddt_attn_args& a = d->attn;
+  ddt_status st = check_attn_args(&a);
+  if (st != DDT_OK) return st;
+  if (d->depth_levels < 1 || d->topk < 1) return DDT_ERR_INVALID_ARG;
+  if (a.B == 0) return DDT_OK;
+  if (!d->lp || !d->tok || !d->root_token || !d->block_ckv || !d->block_krope ||
+      !d->target_continuation || !d->parents || !d->node_tokens || !d->depth ||
+      !d->next_token || !d->next_sibling || !d->target_tokens || !d->path || !d->accept_len)
+    return DDT_ERR_INVALID_ARG;
+  if (!aligned16(d->block_ckv) || !aligned16(d->block_krope)) return DDT_ERR_INVALID_ARG;
+  const int B = a.B, Q = a.q_len;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* row[4] = {nullptr, nullptr, nullptr, nullptr};
+  if (d->status)
+    for (int k = 0; k < 4; ++k) row[k] = d->status + static_cast<int64_t>(k) * B;
+  uint64_t* mask = const_cast<uint64_t*>(a.mask);
+  if (launch_tree_build(d->lp, d->tok, d->root_token, B, d->depth_levels, d->topk, Q, d->parents,
+                        d->node_tokens, d->depth, nullptr, d->next_token, d->next_sibling, mask,
+                        d->n_nodes, row[0], s) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  uint16_t* ckv = static_cast<uint16_t*>(const_cast<void*>(a.c_kv));
+  uint16_t* kr = static_cast<uint16_t*>(const_cast<void*>(a.k_rope));
+  if (launch_kv_write_block(ckv, kr, a.ckv_batch_stride, a.ckv_row_stride, a.kr_batch_stride,
+                            a.kr_row_stride, a.capacity, a.prefix_lens,
+                            static_cast<const uint16_t*>(d->block_ckv),
+                            static_cast<const uint16_t*>(d->block_krope), B, Q, d->depth,
+                            d->target_continuation, d->target_tokens, row[1], s) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  st = ddt_verify_attn(&a, stream);
+  if (st != DDT_OK) return st;
+  if (launch_accept_compact(d->node_tokens, d->target_tokens, d->next_token, d->next_sibling, B,
+                            Q, ckv, kr, a.ckv_batch_stride, a.ckv_row_stride, a.kr_batch_stride,
+                            a.kr_row_stride, a.capacity, a.prefix_lens, d->path, d->accept_len,
+                            d->root_token, row[2], const_cast<int32_t*>(a.prefix_lens), row[3],
+                            s) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  return DDT_OK;
 }
 
 }  // extern "C"

@@ -73,6 +73,40 @@ __global__ void __launch_bounds__(128) build_mask_kernel(const int32_t* __restri
 // ---------------------------------------------------------------------------
 constexpr int kAcceptWarps = 4;
 
+// The walk itself, on one request's arrays in shared memory (one thread).
+// path[0 .. alen) receives the accepted nodes (the caller pre-fills -1);
+// returns the status, with alen and the last accepted node `cur`.
+__device__ int accept_walk(const int32_t* tok, const int32_t* tgt, const int32_t* first,
+                           const int32_t* sib, int q_len, int32_t* path, int& alen, int& cur) {
+  int examined = 0, st = DDT_REQ_OK;
+  alen = 1;
+  cur = 0;
+  path[0] = 0;
+  while (alen < q_len) {
+    int c = first[cur];
+    int found = -1;
+    while (c != -1) {
+      if (c < 0 || c >= q_len) {
+        st = DDT_REQ_BAD_INDEX;
+        break;
+      }
+      if (++examined > q_len) {
+        st = DDT_REQ_WALK_LIMIT;
+        break;
+      }
+      if (tok[c] == tgt[cur]) {
+        found = c;
+        break;
+      }
+      c = sib[c];
+    }
+    if (st != DDT_REQ_OK || found == -1) break;
+    path[alen++] = found;
+    cur = found;
+  }
+  return st;
+}
+
 __global__ void __launch_bounds__(kAcceptWarps * 32) tree_accept_kernel(
     const int32_t* __restrict__ node_tokens, const int32_t* __restrict__ target_tokens,
     const int32_t* __restrict__ next_token, const int32_t* __restrict__ next_sibling, int B,
@@ -97,30 +131,9 @@ __global__ void __launch_bounds__(kAcceptWarps * 32) tree_accept_kernel(
   }
   __syncwarp();
   if (lane == 0) {
-    int alen = 1, cur = 0, examined = 0, st = DDT_REQ_OK;
-    s_path[warp][0] = 0;
-    while (alen < q_len) {
-      int c = s_first[warp][cur];
-      int found = -1;
-      while (c != -1) {
-        if (c < 0 || c >= q_len) {
-          st = DDT_REQ_BAD_INDEX;
-          break;
-        }
-        if (++examined > q_len) {
-          st = DDT_REQ_WALK_LIMIT;
-          break;
-        }
-        if (s_tok[warp][c] == s_tgt[warp][cur]) {
-          found = c;
-          break;
-        }
-        c = s_sib[warp][c];
-      }
-      if (st != DDT_REQ_OK || found == -1) break;
-      s_path[warp][alen++] = found;
-      cur = found;
-    }
+    int alen, cur;
+    const int st = accept_walk(s_tok[warp], s_tgt[warp], s_first[warp], s_sib[warp], q_len,
+                               s_path[warp], alen, cur);
     accept_len[b] = alen;
     if (bonus_token) bonus_token[b] = s_tgt[warp][cur];
     if (status) status[b] = st;
@@ -144,17 +157,47 @@ constexpr int kLatVec = DDT_D_LATENT * 2 / 16;  // 16-byte vectors per latent ro
 constexpr int kRopeVec = DDT_D_ROPE * 2 / 16;   // per rope row (8)
 constexpr int kRowVec = kLatVec + kRopeVec;
 
+// Moves rows P+keep[i] -> P+i (i < alen) of request b, both caches, through
+// shared memory: every moving row is read before any is written.  Called by all
+// kCompactThreads threads of the CTA; s_rows holds alen * kRowVec vectors.
+__device__ void compact_rows(uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope,
+                             int64_t ckv_bs, int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs, int b,
+                             int P, int alen, const int32_t* s_keep, uint4* s_rows) {
+  const uint4* ckv_b = reinterpret_cast<const uint4*>(c_kv + b * ckv_bs);
+  const uint4* kr_b = reinterpret_cast<const uint4*>(k_rope + b * kr_bs);
+  const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;  // row strides in 16-byte vectors
+  const int total = alen * kRowVec;
+  // Phase 1: every moving row into shared memory.
+  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
+    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    if (s_keep[i] == i) continue;
+    const int64_t src_row = P + s_keep[i];
+    s_rows[idx] = (v < kLatVec) ? ckv_b[src_row * ckv_rv + v] : kr_b[src_row * kr_rv + (v - kLatVec)];
+  }
+  __syncthreads();
+  // Phase 2: write rows P .. P+alen-1 (only those that move).
+  uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
+  uint4* kr_w = reinterpret_cast<uint4*>(k_rope + b * kr_bs);
+  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
+    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    if (s_keep[i] == i) continue;
+    const int64_t dst_row = P + i;
+    if (v < kLatVec) ckv_w[dst_row * ckv_rv + v] = s_rows[idx];
+    else kr_w[dst_row * kr_rv + (v - kLatVec)] = s_rows[idx];
+  }
+}
+
 __global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
     uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
-    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* __restrict__ prefix_lens,
+    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* prefix_lens,
     const int32_t* __restrict__ path, const int32_t* __restrict__ accept_len, int q_len,
-    int32_t* __restrict__ new_prefix_lens, int32_t* __restrict__ status) {
+    int32_t* new_prefix_lens, int32_t* __restrict__ status) {
   extern __shared__ uint4 s_rows[];  // [alen][kRowVec]
   __shared__ int32_t s_keep[DDT_MAX_Q_LEN];
   __shared__ int s_state;  // 0 ok, else status code
   const int b = blockIdx.x;
-  const int P = prefix_lens[b];
-  const int alen = accept_len[b];
+  const int P = prefix_lens[b];  // read by every thread before the first barrier, so
+  const int alen = accept_len[b];  // new_prefix_lens may be prefix_lens itself
   if (threadIdx.x == 0) {
     int st = DDT_REQ_OK;
     if (alen < 1 || alen > q_len) st = DDT_REQ_BAD_LENGTH;
@@ -180,31 +223,109 @@ __global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
     }
     return;
   }
-  const uint4* ckv_b = reinterpret_cast<const uint4*>(c_kv + b * ckv_bs);
-  const uint4* kr_b = reinterpret_cast<const uint4*>(k_rope + b * kr_bs);
-  const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;  // row strides in 16-byte vectors
-  const int total = alen * kRowVec;
-  // Phase 1: every moving row into shared memory.
-  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
-    const int i = idx / kRowVec, v = idx - i * kRowVec;
-    if (s_keep[i] == i) continue;
-    const int64_t src_row = P + s_keep[i];
-    s_rows[idx] = (v < kLatVec) ? ckv_b[src_row * ckv_rv + v] : kr_b[src_row * kr_rv + (v - kLatVec)];
-  }
-  __syncthreads();
-  // Phase 2: write rows P .. P+alen-1 (only those that move).
-  uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
-  uint4* kr_w = reinterpret_cast<uint4*>(k_rope + b * kr_bs);
-  for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
-    const int i = idx / kRowVec, v = idx - i * kRowVec;
-    if (s_keep[i] == i) continue;
-    const int64_t dst_row = P + i;
-    if (v < kLatVec) ckv_w[dst_row * ckv_rv + v] = s_rows[idx];
-    else kr_w[dst_row * kr_rv + (v - kLatVec)] = s_rows[idx];
-  }
+  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_keep, s_rows);
   if (threadIdx.x == 0) {
     if (status) status[b] = DDT_REQ_OK;
     if (new_prefix_lens) new_prefix_lens[b] = P + alen;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Accept fused with compaction.  [Race Conditions] "Race Conditions, Buffer
+// Aliasing, ..." closes with the compaction gather as a separate step and names
+// fusing it as later work.  Here one CTA per request walks the tree (thread 0,
+// the same walk as tree_accept_kernel) and then moves the accepted rows (all
+// threads, the same staging as kv_compact_kernel), so the path never leaves the
+// chip and one launch replaces two.  The walk always yields 1 <= alen <= q_len
+// and path entries in [0, q_len), so compaction can only fail on the prefix.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCompactThreads) accept_compact_kernel(
+    const int32_t* __restrict__ node_tokens, const int32_t* __restrict__ target_tokens,
+    const int32_t* __restrict__ next_token, const int32_t* __restrict__ next_sibling, int q_len,
+    uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
+    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* prefix_lens,
+    int32_t* __restrict__ path, int32_t* __restrict__ accept_len, int32_t* __restrict__ bonus_token,
+    int32_t* __restrict__ accept_status, int32_t* new_prefix_lens,
+    int32_t* __restrict__ compact_status) {
+  extern __shared__ uint4 s_rows[];  // [alen][kRowVec]
+  __shared__ int32_t s_tok[DDT_MAX_Q_LEN], s_tgt[DDT_MAX_Q_LEN], s_first[DDT_MAX_Q_LEN],
+      s_sib[DDT_MAX_Q_LEN], s_path[DDT_MAX_Q_LEN];
+  __shared__ int s_alen, s_state;
+  const int b = blockIdx.x;
+  const int P = prefix_lens[b];  // read by every thread before the first barrier
+  const int64_t base = static_cast<int64_t>(b) * q_len;
+  for (int k = threadIdx.x; k < q_len; k += kCompactThreads) {
+    s_tok[k] = node_tokens[base + k];
+    s_tgt[k] = target_tokens[base + k];
+    s_first[k] = next_token[base + k];
+    s_sib[k] = next_sibling[base + k];
+    s_path[k] = -1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int alen, cur;
+    const int st = accept_walk(s_tok, s_tgt, s_first, s_sib, q_len, s_path, alen, cur);
+    accept_len[b] = alen;
+    if (bonus_token) bonus_token[b] = s_tgt[cur];
+    if (accept_status) accept_status[b] = st;
+    s_alen = alen;
+    s_state = (P < 0 || static_cast<int64_t>(P) + q_len > capacity) ? DDT_REQ_BAD_PREFIX
+                                                                     : DDT_REQ_OK;
+  }
+  __syncthreads();
+  const int alen = s_alen;
+  for (int k = threadIdx.x; k < q_len; k += kCompactThreads) path[base + k] = s_path[k];
+  if (s_state != DDT_REQ_OK) {
+    if (threadIdx.x == 0) {
+      if (compact_status) compact_status[b] = s_state;
+      if (new_prefix_lens) new_prefix_lens[b] = P;
+    }
+    return;
+  }
+  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_path, s_rows);
+  if (threadIdx.x == 0) {
+    if (compact_status) compact_status[b] = DDT_REQ_OK;
+    if (new_prefix_lens) new_prefix_lens[b] = P + alen;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tree-block write.  [Race Conditions] "The Cache Compaction Problem": the tree
+// block's KV rows go into the cache right after the prefix, node i at row P+i
+// (absolute positions offset by the prefix length).  One CTA per request copies
+// the q_len rows (latent and rope) with 16-byte vectors.  Optionally, as the
+// stand-in for the target model's greedy tokens, target_tokens[b,i] is taken
+// from a per-depth continuation: cont[b, depth[b,i]] (the target's greedy token
+// after the accepted prefix of that depth).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kCompactThreads) kv_write_block_kernel(
+    uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
+    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* __restrict__ prefix_lens,
+    const uint16_t* __restrict__ block_ckv, const uint16_t* __restrict__ block_krope, int q_len,
+    const int32_t* __restrict__ depth, const int32_t* __restrict__ cont,
+    int32_t* __restrict__ target_tokens, int32_t* __restrict__ status) {
+  const int b = blockIdx.x;
+  const int P = prefix_lens[b];
+  const bool ok = P >= 0 && static_cast<int64_t>(P) + q_len <= capacity;
+  const int64_t base = static_cast<int64_t>(b) * q_len;
+  if (cont) {
+    for (int i = threadIdx.x; i < q_len; i += kCompactThreads) {
+      const int d = depth[base + i];
+      target_tokens[base + i] = (d >= 0 && d < q_len) ? cont[base + d] : -1;
+    }
+  }
+  if (threadIdx.x == 0 && status) status[b] = ok ? DDT_REQ_OK : DDT_REQ_BAD_PREFIX;
+  if (!ok) return;
+  const uint4* src_l = reinterpret_cast<const uint4*>(block_ckv) + base * kLatVec;
+  const uint4* src_r = reinterpret_cast<const uint4*>(block_krope) + base * kRopeVec;
+  uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
+  uint4* kr_w = reinterpret_cast<uint4*>(k_rope + b * kr_bs);
+  const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;
+  for (int idx = threadIdx.x; idx < q_len * kRowVec; idx += kCompactThreads) {
+    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    const int64_t row = P + i;
+    if (v < kLatVec) ckv_w[row * ckv_rv + v] = src_l[static_cast<int64_t>(i) * kLatVec + v];
+    else kr_w[row * kr_rv + (v - kLatVec)] = src_r[static_cast<int64_t>(i) * kRopeVec + (v - kLatVec)];
   }
 }
 
@@ -240,6 +361,36 @@ cudaError_t launch_kv_compact(uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs, 
   kv_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
       c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, capacity, prefix_lens, path, accept_len, q_len,
       new_prefix_lens, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_accept_compact(const int32_t* node_tokens, const int32_t* target_tokens,
+                                  const int32_t* next_token, const int32_t* next_sibling, int B,
+                                  int q_len, uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs,
+                                  int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs, int capacity,
+                                  const int32_t* prefix_lens, int32_t* path, int32_t* accept_len,
+                                  int32_t* bonus, int32_t* accept_status, int32_t* new_prefix_lens,
+                                  int32_t* compact_status, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(q_len) * kRowVec * sizeof(uint4);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(accept_compact_kernel),
+                                    static_cast<int>(DDT_MAX_Q_LEN * kRowVec * sizeof(uint4)), 4);
+  if (e != cudaSuccess) return e;
+  accept_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
+      node_tokens, target_tokens, next_token, next_sibling, q_len, c_kv, k_rope, ckv_bs, ckv_rs,
+      kr_bs, kr_rs, capacity, prefix_lens, path, accept_len, bonus, accept_status,
+      new_prefix_lens, compact_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_write_block(uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs,
+                                  int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs, int capacity,
+                                  const int32_t* prefix_lens, const uint16_t* block_ckv,
+                                  const uint16_t* block_krope, int B, int q_len,
+                                  const int32_t* depth, const int32_t* cont,
+                                  int32_t* target_tokens, int32_t* status, cudaStream_t stream) {
+  kv_write_block_kernel<<<B, kCompactThreads, 0, stream>>>(
+      c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, capacity, prefix_lens, block_ckv, block_krope,
+      q_len, depth, cont, target_tokens, status);
   return cudaGetLastError();
 }
 

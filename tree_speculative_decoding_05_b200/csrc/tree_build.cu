@@ -1,0 +1,236 @@
+// tree_build.cu — best-first draft-tree construction on the GPU.
+//
+// Sources (page title, section):
+//   [Foundation] "Building the Foundation: Architecting a Native CUDA DDTree
+//       Inference Engine": "The Single-Threaded Heap Design" (one serial
+//       best-first expansion per request, budget <= 64 and depth <= 15 small
+//       enough for on-chip memory, the other threads of the block build the
+//       visibility rows and retrieve pointers), "Tie-Breaking and Numerical
+//       Precision" (equal weights in insertion order, float32 arithmetic),
+//       "Assumptions Underlying the Design" (item 4: the sibling weight is the
+//       parent-relative expression logw - lp[depth-1][rank] + lp[depth-1][rank+1]
+//       evaluated in that order; item 5: candidates can run out before the
+//       budget when topk is 1).
+//
+// The expansion (per request; rows d of lp / tok describe tree depth d+1):
+//   node 0 = root (depth 0, logw 0, parent -1, the root token);
+//   candidates start with (0 + lp[0][0], depth 1, rank 0, parent 0);
+//   while fewer than q_len nodes and a candidate remains: the candidate of
+//   largest logw (earliest inserted among equals) becomes the next node n with
+//   token tok[d-1][r]; then insert its first child (logw + lp[d][0], d+1, 0, n)
+//   if d < D, then its next sibling ((logw - lp[d-1][r]) + lp[d-1][r+1], d,
+//   r+1, parent) if r+1 < K.
+//
+// B200 design.  The expansion is serial in its picks but each pick is a max
+// over at most 2*q_len candidates, so one warp per request keeps the candidate
+// list in registers (slot s lives in lane s % 32, register s / 32; slots are
+// handed out in insertion order, so the slot number is the tie-break key) and
+// takes every pick with one warp-wide arg-max of (logw, slot) — five shuffle
+// rounds, no heap and no shared-memory round trip.  The log-probs and tokens a
+// build can touch (depth rows < min(D, q_len-1), ranks < min(K, q_len)) are
+// staged in shared memory first, so no pick waits on global memory.  The
+// weights use explicitly rounded float32 adds and subtracts (__fadd_rn /
+// __fsub_rn), which the compiler may neither contract nor reorder, so the
+// result is bit-identical to any float32 evaluation of the same expressions.
+// After the expansion the lanes build, one node each, the visibility words,
+// the retrieve pointers and the padding, and write everything coalesced.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "ddt.h"
+#include "ddt_internal.h"
+
+namespace ddt {
+
+namespace tb {
+constexpr int kSlotRegs = 2 * DDT_MAX_Q_LEN / 32;  // 2*q_len - 1 insertions at most
+// Dynamic shared memory bound: rows < q_len-1, ranks < q_len, float + int each.
+constexpr int kMaxStageBytes = (DDT_MAX_Q_LEN - 1) * DDT_MAX_Q_LEN * 8;
+}  // namespace tb
+
+__global__ void __launch_bounds__(32) tree_build_kernel(
+    const float* __restrict__ lp, const int32_t* __restrict__ tok,
+    const int32_t* __restrict__ root_token, int D, int K, int q_len, int Dp, int Kp,
+    int32_t* __restrict__ parents, int32_t* __restrict__ node_tokens, int32_t* __restrict__ depth,
+    float* __restrict__ logw, int32_t* __restrict__ next_token,
+    int32_t* __restrict__ next_sibling, uint64_t* __restrict__ mask,
+    int32_t* __restrict__ n_nodes, int32_t* __restrict__ status) {
+  using namespace tb;
+  extern __shared__ __align__(16) unsigned char tb_smem[];
+  float* s_lp = reinterpret_cast<float*>(tb_smem);                   // [Dp][Kp]
+  int32_t* s_tok = reinterpret_cast<int32_t*>(tb_smem) + Dp * Kp;   // [Dp][Kp]
+  __shared__ int32_t s_par[DDT_MAX_Q_LEN];
+  __shared__ int32_t s_ntok[DDT_MAX_Q_LEN];
+  __shared__ int32_t s_dep[DDT_MAX_Q_LEN];
+  __shared__ float s_lw[DDT_MAX_Q_LEN];
+
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int64_t DK = static_cast<int64_t>(D) * K;
+  const float* L = lp + b * DK;
+  const int32_t* T = tok + b * DK;
+
+  // Every log-prob must be finite (a NaN would make the arg-max order-dependent).
+  bool bad = false;
+  for (int64_t e = lane; e < DK; e += 32) bad |= !isfinite(L[e]);
+  bad = __any_sync(0xffffffffu, bad);
+
+  for (int e = lane; e < Dp * Kp; e += 32) {
+    const int d = e / Kp, r = e - d * Kp;
+    s_lp[e] = L[static_cast<int64_t>(d) * K + r];
+    s_tok[e] = T[static_cast<int64_t>(d) * K + r];
+  }
+  if (lane == 0) {
+    s_par[0] = -1;
+    s_ntok[0] = root_token[b];
+    s_dep[0] = 0;
+    s_lw[0] = 0.0f;
+  }
+  __syncwarp();
+
+  // Candidate slots: weight and packed (depth | rank << 8 | parent << 16); -1 = empty.
+  float cw[kSlotRegs];
+  int cm[kSlotRegs];
+#pragma unroll
+  for (int j = 0; j < kSlotRegs; ++j) {
+    cw[j] = -INFINITY;
+    cm[j] = -1;
+  }
+  int n_slots = 0;
+  auto insert = [&](float w, int meta) {
+    const int s = n_slots++;
+#pragma unroll
+    for (int j = 0; j < kSlotRegs; ++j)
+      if (j == (s >> 5) && lane == (s & 31)) {
+        cw[j] = w;
+        cm[j] = meta;
+      }
+  };
+  if (!bad && q_len > 1) insert(__fadd_rn(0.0f, s_lp[0]), 1 | (0 << 8) | (0 << 16));
+
+  int n = 1;
+  while (n < q_len) {
+    // Lane-local best: slots ascend with j, so a later equal weight never wins.
+    float bw = -INFINITY;
+    int bs = INT_MAX;
+#pragma unroll
+    for (int j = 0; j < kSlotRegs; ++j)
+      if (cm[j] >= 0 && (cw[j] > bw || bs == INT_MAX)) {
+        bw = cw[j];
+        bs = j * 32 + lane;
+      }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ow = __shfl_xor_sync(0xffffffffu, bw, off);
+      const int os = __shfl_xor_sync(0xffffffffu, bs, off);
+      if (os != INT_MAX && (bs == INT_MAX || ow > bw || (ow == bw && os < bs))) {
+        bw = ow;
+        bs = os;
+      }
+    }
+    if (bs == INT_MAX) break;  // no candidate left
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < kSlotRegs; ++j)
+      if (j == (bs >> 5) && lane == (bs & 31)) {
+        mine = cm[j];
+        cm[j] = -1;
+      }
+    const int meta = __shfl_sync(0xffffffffu, mine, bs & 31);
+    const int d = meta & 0xff, r = (meta >> 8) & 0xff, par = meta >> 16;
+    const int node = n++;
+    if (lane == 0) {
+      s_par[node] = par;
+      s_ntok[node] = s_tok[(d - 1) * Kp + r];
+      s_dep[node] = d;
+      s_lw[node] = bw;
+    }
+    if (n == q_len) break;  // budget reached: nothing more will be picked
+    if (d < D) insert(__fadd_rn(bw, s_lp[d * Kp]), (d + 1) | (0 << 8) | (node << 16));
+    if (r + 1 < K) {
+      const float w = __fadd_rn(__fsub_rn(bw, s_lp[(d - 1) * Kp + r]), s_lp[(d - 1) * Kp + r + 1]);
+      insert(w, d | ((r + 1) << 8) | (par << 16));
+    }
+  }
+  __syncwarp();
+
+  // Per node: padding, retrieve pointers, visibility words; coalesced writes.
+  const int W = (q_len + 63) >> 6;
+  const int64_t row0 = static_cast<int64_t>(b) * q_len;
+  for (int i = lane; i < q_len; i += 32) {
+    int p, t, dd, first = -1, sib = -1;
+    float w;
+    uint64_t w0 = 0, w1 = 0;
+    if (i < n) {
+      p = s_par[i];
+      t = s_ntok[i];
+      dd = s_dep[i];
+      w = s_lw[i];
+      for (int c = i + 1; c < n; ++c)
+        if (s_par[c] == i) {
+          first = c;
+          break;
+        }
+      if (i > 0)
+        for (int c = i + 1; c < n; ++c)
+          if (s_par[c] == p) {
+            sib = c;
+            break;
+          }
+      for (int a = i, steps = 0; a >= 0 && steps <= i; a = s_par[a], ++steps) {
+        if (a < 64) w0 |= 1ull << a;
+        else w1 |= 1ull << (a - 64);
+      }
+    } else {
+      p = 0;
+      t = -1;
+      dd = 1;
+      w = -INFINITY;
+      w0 = 1ull;
+      if (i < 64) w0 |= 1ull << i;
+      else w1 |= 1ull << (i - 64);
+    }
+    parents[row0 + i] = p;
+    node_tokens[row0 + i] = t;
+    next_token[row0 + i] = first;
+    next_sibling[row0 + i] = sib;
+    if (depth) depth[row0 + i] = dd;
+    if (logw) logw[row0 + i] = w;
+    if (mask) {
+      uint64_t* m = mask + (row0 + i) * W;
+      m[0] = w0;
+      if (W > 1) m[1] = w1;
+    }
+  }
+  if (lane == 0) {
+    if (n_nodes) n_nodes[b] = n;
+    if (status) status[b] = bad ? DDT_REQ_BAD_LP : DDT_REQ_OK;
+  }
+}
+
+size_t tree_build_smem_bytes(int D, int K, int q_len) {
+  const int Dp = D < q_len - 1 ? D : q_len - 1;
+  const int Kp = K < q_len ? K : q_len;
+  return static_cast<size_t>(Dp > 0 ? Dp : 0) * static_cast<size_t>(Kp) * 8;
+}
+
+cudaError_t launch_tree_build(const float* lp, const int32_t* tok, const int32_t* root_token,
+                              int B, int D, int K, int q_len, int32_t* parents,
+                              int32_t* node_tokens, int32_t* depth, float* logw,
+                              int32_t* next_token, int32_t* next_sibling, uint64_t* mask,
+                              int32_t* n_nodes, int32_t* status, cudaStream_t stream) {
+  const int Dp = D < q_len - 1 ? D : q_len - 1;
+  const int Kp = K < q_len ? K : q_len;
+  const size_t smem = tree_build_smem_bytes(D, K, q_len);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(tree_build_kernel),
+                                    tb::kMaxStageBytes, 3);
+  if (e != cudaSuccess) return e;
+  tree_build_kernel<<<B, 32, smem, stream>>>(lp, tok, root_token, D, K, q_len, Dp > 0 ? Dp : 0,
+                                             Kp, parents, node_tokens, depth, logw, next_token,
+                                             next_sibling, mask, n_nodes, status);
+  return cudaGetLastError();
+}
+
+}  // namespace ddt

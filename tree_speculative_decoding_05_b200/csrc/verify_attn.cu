@@ -44,6 +44,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -128,6 +129,11 @@ struct VerifyParams {
   int32_t* status;
   int B, Q, capacity, num_splits, n_pairs, out_f32;
   float scale_log2;  // softmax_scale * log2(e)
+  // Key range of a launch: 0 = the whole cache (prefix and tree block); 1 = the
+  // prefix rows [0, P) only; 2 = the tree block [P, P+Q) only (one tile).
+  int kv_mode;
+  int write_partials;  // write normalised partials + lse (split-KV or a pass of a split)
+  int split_base;      // partial index of this launch's split 0
 };
 
 // KV tile range [t0, t1) of split `split` for a cache of T rows.
@@ -140,7 +146,7 @@ __host__ __device__ inline void split_range(int T, int num_splits, int split, in
 
 // One work item: a pair of tree nodes of one request over one KV split.
 struct WorkItem {
-  int b, pair, split, P, T, t0, ntile, last_tile;
+  int b, pair, split, P, T, end, t0, ntile, last_tile;  // end: last row + 1 of this pass
   bool bad_prefix, valid;
 };
 
@@ -158,21 +164,29 @@ __device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int w, co
   // Requests whose tree block would not fit the cache are rejected as a whole.
   it.bad_prefix = (it.P < 0) || (static_cast<int64_t>(it.P) + p.Q > p.capacity);
   it.T = it.P + p.Q;
+  it.end = p.kv_mode == 1 ? it.P : it.T;
   int t0 = 0, t1 = 0;
-  if (!it.bad_prefix) split_range(it.T, p.num_splits, it.split, t0, t1);
+  if (!it.bad_prefix) {
+    if (p.kv_mode == 2) {
+      t0 = (it.T + 127) / 128 - 1;  // the one tile ending at T holds the tree block (Q <= 128)
+      t1 = t0 + 1;
+    } else {
+      split_range(it.end, p.num_splits, it.split, t0, t1);
+    }
+  }
   it.t0 = t0;
   it.ntile = t1 - t0;  // 0 for an empty split (the merge skips it)
-  it.last_tile = (it.T + 127) / 128 - 1;
+  it.last_tile = (it.end + 127) / 128 - 1;
   it.valid = !it.bad_prefix && it.ntile > 0;
   return it;
 }
 
-// First cache row of KV tile t.  A request's last tile is shifted to end at row
-// T, so no load ever reaches the rows past the tree block (padding that may hold
-// anything); its overlap with the previous tile is masked, and rows below 0
-// (T < 128) read as zeros.
+// First cache row of KV tile t.  A request's last tile is shifted to end at the
+// pass's last row (T, or P for a prefix pass), so no load ever reaches the rows
+// past it (padding that may hold anything); its overlap with the previous tile
+// is masked, and rows below 0 (fewer than 128 rows) read as zeros.
 __device__ __forceinline__ int tile_start(const WorkItem& it, int t) {
-  return t == it.last_tile ? it.T - 128 : 128 * t;
+  return t == it.last_tile ? it.end - 128 : 128 * t;
 }
 
 // The k-th work index of a cluster: rounds of n_clusters indices, alternating
@@ -518,13 +532,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
         }
         const int key0 = tile_start(it, tile) + hf * 64;
-        const int lo = tile * 128;  // keys below lo belong to the previous tile
-        if (key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
+        // Keys below lo belong to the previous tile (a tree-block pass has none).
+        // Prefix rows are visible to every node, except in a tree-block pass,
+        // whose one tile may also reach prefix rows and rows below 0.
+        const bool tree_pass = p.kv_mode == 2;
+        const int lo = tree_pass ? INT_MIN : tile * 128;
+        if (tree_pass || key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             const int key = key0 + c;
-            bool vis = key < P;
-            if (!vis && key < T) {
+            bool vis = !tree_pass && key < P;
+            if (!vis && key >= P && key < T) {
               const int a = key - P;
               const uint64_t w = a < 64 ? mw0 : mw1;
               vis = (w >> (a & 63)) & 1ull;
@@ -613,9 +631,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
             tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
             tmem_wait_ld();
             const int col = 256 * nh + 128 * hf + 32 * q;
-            if (p.num_splits > 1) {
+            if (p.write_partials) {
               float4* dst = reinterpret_cast<float4*>(
-                  p.part_o + (static_cast<int64_t>(split) * rows_total + row) * 512 + col);
+                  p.part_o + (static_cast<int64_t>(split + p.split_base) * rows_total + row) * 512 +
+                  col);
 #pragma unroll
               for (int v = 0; v < 8; ++v)
                 dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
@@ -641,7 +660,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           }
         }
         if (hf == 0) {
-          if (p.num_splits > 1) p.part_lse[static_cast<int64_t>(split) * rows_total + row] = lse_nat;
+          if (p.write_partials)
+            p.part_lse[static_cast<int64_t>(split + p.split_base) * rows_total + row] = lse_nat;
           else if (p.lse) p.lse[row] = lse_nat;
         }
       }
@@ -669,7 +689,8 @@ __global__ void __launch_bounds__(256) verify_merge_kernel(const float* __restri
                                                            const int32_t* __restrict__ prefix_lens,
                                                            void* __restrict__ out, int out_f32,
                                                            float* __restrict__ lse, int B, int Q,
-                                                           int capacity, int num_splits) {
+                                                           int capacity, int num_splits,
+                                                           int tail) {
   const int64_t rows_total = static_cast<int64_t>(B) * Q * 64;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -677,21 +698,25 @@ __global__ void __launch_bounds__(256) verify_merge_kernel(const float* __restri
   const int b = static_cast<int>(row / (static_cast<int64_t>(Q) * 64));
   const int P = prefix_lens[b];
   if (P < 0 || static_cast<int64_t>(P) + Q > capacity) return;
-  const int T = P + Q;
-  float lmax = -INFINITY;
-  int ns = 0;
-  for (int s = 0; s < num_splits; ++s) {
+  // Partials present: the non-empty splits of the cache (whole, or with `tail`
+  // the prefix rows [0, P) in num_splits - 1 splits), then the tree block's.
+  const int T = tail ? P : P + Q;
+  const int n_cache = tail ? num_splits - 1 : num_splits;
+  auto present = [&](int s) {
+    if (s >= n_cache) return true;  // the tree-block partial
     int t0, t1;
-    split_range(T, num_splits, s, t0, t1);
-    if (t0 >= t1) break;
-    ns = s + 1;
-    lmax = fmaxf(lmax, part_lse[s * rows_total + row]);
-  }
+    split_range(T, n_cache, s, t0, t1);
+    return t0 < t1;
+  };
+  float lmax = -INFINITY;
+  for (int s = 0; s < num_splits; ++s)
+    if (present(s)) lmax = fmaxf(lmax, part_lse[s * rows_total + row]);
   float acc[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) acc[k] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < ns; ++s) {
+  for (int s = 0; s < num_splits; ++s) {
+    if (!present(s)) continue;
     const float ls = part_lse[s * rows_total + row];
     const float w = (ls == -INFINITY) ? 0.f : fast_exp2((ls - lmax) * va::kLog2e);
     wsum += w;
@@ -796,8 +821,11 @@ size_t verify_workspace_bytes(const ddt_attn_args& a, int num_splits) {
   return static_cast<size_t>(num_splits) * rows * (512 + 1) * sizeof(float);
 }
 
-ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* part_o,
-                              float* part_lse, cudaStream_t stream) {
+namespace {
+
+// One launch of the verify kernel over key range `kv_mode` (see VerifyParams).
+ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int write_partials,
+                       int split_base, float* part_o, float* part_lse, cudaStream_t stream) {
   using namespace va;
   CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope;
   const uint64_t rows_q = static_cast<uint64_t>(a.q_len) * 64;
@@ -827,6 +855,9 @@ ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* par
   p.n_pairs = (a.q_len + 1) / 2;
   p.out_f32 = a.out_dtype == DDT_F32;
   p.scale_log2 = a.softmax_scale * kLog2e;
+  p.kv_mode = kv_mode;
+  p.write_partials = write_partials;
+  p.split_base = split_base;
   // Persistent grid: at most one CTA pair per two SMs; pairs loop over items.
   const int64_t items = static_cast<int64_t>(a.B) * p.n_pairs * num_splits;
   if (items > 0x3fffffffll) return DDT_ERR_UNSUPPORTED;
@@ -834,15 +865,35 @@ ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* par
   const int64_t grid = 2 * (items < slots ? items : slots);
   verify_attn_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
       m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, p);
-  if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
-  if (num_splits > 1) {
-    const int64_t rows = static_cast<int64_t>(a.B) * a.q_len * 64;
-    verify_merge_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-        part_o, part_lse, a.prefix_lens, a.out, p.out_f32, a.lse, a.B, a.q_len, a.capacity,
-        num_splits);
-    if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
-  }
-  return DDT_OK;
+  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+}
+
+ddt_status launch_merge(const ddt_attn_args& a, int num_partials, int tail, const float* part_o,
+                        const float* part_lse, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(a.B) * a.q_len * 64;
+  verify_merge_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      part_o, part_lse, a.prefix_lens, a.out, a.out_dtype == DDT_F32, a.lse, a.B, a.q_len,
+      a.capacity, num_partials, tail);
+  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+}
+
+}  // namespace
+
+ddt_status launch_verify_attn(const ddt_attn_args& a, int num_splits, float* part_o,
+                              float* part_lse, cudaStream_t stream) {
+  const ddt_status st =
+      launch_pass(a, 0, num_splits, num_splits > 1, 0, part_o, part_lse, stream);
+  if (st != DDT_OK || num_splits <= 1) return st;
+  return launch_merge(a, num_splits, 0, part_o, part_lse, stream);
+}
+
+ddt_status launch_verify_attn_split_tail(const ddt_attn_args& a, int prefix_splits,
+                                         float* part_o, float* part_lse, cudaStream_t stream) {
+  ddt_status st = launch_pass(a, 1, prefix_splits, 1, 0, part_o, part_lse, stream);
+  if (st != DDT_OK) return st;
+  st = launch_pass(a, 2, 1, 1, prefix_splits, part_o, part_lse, stream);
+  if (st != DDT_OK) return st;
+  return launch_merge(a, prefix_splits + 1, 1, part_o, part_lse, stream);
 }
 
 }  // namespace ddt

@@ -35,6 +35,7 @@ VOCAB = 32000
 
 # Stream tags: each array draws from its own stream of the request's seed.
 TAG_PARENTS, TAG_QLAT, TAG_QROPE, TAG_CKV, TAG_KROPE, TAG_TOKENS, TAG_SCALE, TAG_PREFIX = range(8)
+TAG_DRAFT_LOGITS, TAG_DRAFT_TOKENS = 8, 9
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -308,6 +309,59 @@ def make_workload(name: str, seed: int, B: int, q_len: int, prefix_lens, *,
                     node_tokens=node_tokens, target_tokens=target, next_token=nt, next_sibling=ns,
                     softmax_scale=float(np.float32(1.0 / math.sqrt(192.0))), out_dtype=out_dtype,
                     want_lse=want_lse, forced_path=np.stack(forced) if forced else None)
+
+
+@dataclasses.dataclass
+class DraftBatch:
+    """Per-depth top-k draft distributions of a batch: lp float32 [B, D, K] (log-
+    probabilities, each row descending), tok int32 [B, D, K] (distinct per row),
+    root_token int32 [B]."""
+    lp: np.ndarray
+    tok: np.ndarray
+    root_token: np.ndarray
+
+
+def draft_batch(seed: int, B: int, D: int, K: int, *, vocab: int = VOCAB,
+                temperature: float = 8.0, quantum: float = 0.0, sort: bool = True) -> DraftBatch:
+    """Synthetic drafter output.  Row (b, d) has K logits z ~ N(0, 1) * temperature
+    and one tail logit ln(vocab - K) standing for the rest of the vocabulary (each of
+    its tokens at logit 0); lp is the log-softmax of the K head logits over all
+    K + 1, rounded to float32 and sorted descending.  quantum > 0 rounds lp to
+    multiples of quantum (to force equal weights); sort=False keeps draw order."""
+    z = normal(stream_base(seed, TAG_DRAFT_LOGITS, 0), B * D * K).reshape(B, D, K) * temperature
+    tail = math.log(vocab - K)
+    m = np.maximum(z.max(axis=2, keepdims=True), tail)
+    lse = m + np.log(np.exp(z - m).sum(axis=2, keepdims=True) + np.exp(tail - m))
+    lp = z - lse
+    if quantum > 0:
+        lp = np.round(lp / quantum) * quantum
+    if sort:
+        lp = -np.sort(-lp, axis=2)
+    tok = np.zeros((B, D, K), dtype=np.int32)
+    roots = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        r = raw_u64(stream_base(seed, TAG_DRAFT_TOKENS, b), 0, 1 + D * K)
+        roots[b] = int(r[0] % np.uint64(vocab))
+        for d in range(D):
+            row: list[int] = []
+            for x in r[1 + d * K: 1 + (d + 1) * K]:
+                t = int(x % np.uint64(vocab))
+                while t in row:  # distinct within a row
+                    t = (t + 1) % vocab
+                row.append(t)
+            tok[b, d] = row
+    return DraftBatch(lp=lp.astype(np.float32), tok=tok, root_token=roots)
+
+
+def subset(w: Workload, idx) -> Workload:
+    """The requests `idx` of a workload (every per-request array sliced alike)."""
+    idx = np.asarray(idx, dtype=np.int64)
+    per_request = ("prefix_lens", "parents", "q_lat", "q_rope", "c_kv", "k_rope", "node_tokens",
+                   "target_tokens", "next_token", "next_sibling")
+    kw = {k: np.ascontiguousarray(getattr(w, k)[idx]) for k in per_request}
+    if w.forced_path is not None:
+        kw["forced_path"] = np.ascontiguousarray(w.forced_path[idx])
+    return dataclasses.replace(w, B=int(len(idx)), **kw)
 
 
 def ragged_prefixes(seed: int, B: int, lo: int, hi: int) -> np.ndarray:
