@@ -43,10 +43,11 @@ def _check(w, rows=None, num_splits=0, what=""):
     compare_attention(rows_of(out, rows), o_ref, what)
     l_gpu = lse.reshape(-1).cpu().numpy()[rows].astype(np.float64)
     assert np.max(np.abs(l_gpu - l_ref)) <= LSE_MAX_ABS, what
-    # and against the fused pass
+    # and against the fused pass: both are within MAX_ABS of the exact values, so
+    # they differ by at most twice that (a bf16 ulp at |o| ~ 7 is already 0.03)
     f_out, f_lse, _ = dw.verify()
     torch.cuda.synchronize()
-    assert float((f_out.float() - out.float()).abs().max()) <= MAX_ABS, what
+    assert float((f_out.float() - out.float()).abs().max()) <= 2 * MAX_ABS, what
 
 
 @pytest.mark.parametrize("Q,P", [(1, 0), (2, 0), (9, 0), (3, 5), (9, 127), (17, 128),

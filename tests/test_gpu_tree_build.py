@@ -61,6 +61,10 @@ def test_tree_build_ties_follow_insertion_order():
     _check(lp, tok, root, 65)
     lp = np.full((4, 6, 4), -1.0, np.float32)  # every weight ties
     _check(lp, tok[:4, :6, :4], root[:4], 40)
+    lp = np.zeros((4, 6, 4), np.float32)  # +0 and -0 weights are equal weights
+    lp[:, :, 1::2] = -0.0
+    lp[1:, 2, :] = np.float32(-0.5)
+    _check(lp, tok[:4, :6, :4], root[:4], 40)
 
 
 def test_tree_build_unsorted_rows():

@@ -23,10 +23,13 @@
 //
 // B200 design.  The expansion is serial in its picks but each pick is a max
 // over at most 2*q_len candidates, so one warp per request keeps the candidate
-// list in registers (slot s lives in lane s % 32, register s / 32; slots are
-// handed out in insertion order, so the slot number is the tie-break key) and
-// takes every pick with one warp-wide arg-max of (logw, slot) — five shuffle
-// rounds, no heap and no shared-memory round trip.  The log-probs and tokens a
+// list spread over its lanes: slot s lives in lane s % 32, register s / 32, and
+// slots are handed out in insertion order, so the slot number is the tie-break
+// key.  A register holds an order-preserving 32-bit key of the weight (larger
+// weight, larger key; equal weights, equal keys; 0 = empty slot); the exact
+// weight and the (depth, rank, parent) of each slot sit in shared memory.  A
+// pick is two warp-wide hardware reductions: the maximum key, then the
+// smallest slot holding it — no heap and no shuffle tree.  The log-probs and tokens a
 // build can touch (depth rows < min(D, q_len-1), ranks < min(K, q_len)) are
 // staged in shared memory first, so no pick waits on global memory.  The
 // weights use explicitly rounded float32 adds and subtracts (__fadd_rn /
@@ -45,10 +48,17 @@
 namespace ddt {
 
 namespace tb {
-constexpr int kSlotRegs = 2 * DDT_MAX_Q_LEN / 32;  // 2*q_len - 1 insertions at most
 // Dynamic shared memory bound: rows < q_len-1, ranks < q_len, float + int each.
 constexpr int kMaxStageBytes = (DDT_MAX_Q_LEN - 1) * DDT_MAX_Q_LEN * 8;
 }  // namespace tb
+
+// Order-preserving key of a weight: larger weight, larger key; -0 and +0 map to
+// the same key; every key of a non-NaN weight is non-zero (0 marks an empty slot).
+__device__ __forceinline__ uint32_t weight_key(float w) {
+  uint32_t u = __float_as_uint(w);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 __global__ void __launch_bounds__(32) tree_build_kernel(
     const float* __restrict__ lp, const int32_t* __restrict__ tok,
@@ -57,7 +67,6 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     float* __restrict__ logw, int32_t* __restrict__ next_token,
     int32_t* __restrict__ next_sibling, uint64_t* __restrict__ mask,
     int32_t* __restrict__ n_nodes, int32_t* __restrict__ status) {
-  using namespace tb;
   extern __shared__ __align__(16) unsigned char tb_smem[];
   float* s_lp = reinterpret_cast<float*>(tb_smem);                   // [Dp][Kp]
   int32_t* s_tok = reinterpret_cast<int32_t*>(tb_smem) + Dp * Kp;   // [Dp][Kp]
@@ -65,6 +74,9 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   __shared__ int32_t s_ntok[DDT_MAX_Q_LEN];
   __shared__ int32_t s_dep[DDT_MAX_Q_LEN];
   __shared__ float s_lw[DDT_MAX_Q_LEN];
+  __shared__ uint32_t s_ck[2 * DDT_MAX_Q_LEN];  // candidate order key per slot, 0 = empty
+  __shared__ float s_cw[2 * DDT_MAX_Q_LEN];     // candidate weight per slot
+  __shared__ int32_t s_cm[2 * DDT_MAX_Q_LEN];   // candidate depth | rank << 8 | parent << 16
 
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
@@ -90,55 +102,38 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   }
   __syncwarp();
 
-  // Candidate slots: weight and packed (depth | rank << 8 | parent << 16); -1 = empty.
-  float cw[kSlotRegs];
-  int cm[kSlotRegs];
-#pragma unroll
-  for (int j = 0; j < kSlotRegs; ++j) {
-    cw[j] = -INFINITY;
-    cm[j] = -1;
-  }
+  // Candidate slots in insertion order; lane l scans slots l, l + 32, ...
   int n_slots = 0;
-  auto insert = [&](float w, int meta) {
-    const int s = n_slots++;
-#pragma unroll
-    for (int j = 0; j < kSlotRegs; ++j)
-      if (j == (s >> 5) && lane == (s & 31)) {
-        cw[j] = w;
-        cm[j] = meta;
-      }
+  auto insert = [&](float w, int meta) {  // one slot, written by lane 0
+    if (lane == 0) {
+      s_ck[n_slots] = weight_key(w);
+      s_cw[n_slots] = w;
+      s_cm[n_slots] = meta;
+    }
+    ++n_slots;
   };
   if (!bad && q_len > 1) insert(__fadd_rn(0.0f, s_lp[0]), 1 | (0 << 8) | (0 << 16));
+  __syncwarp();
 
   int n = 1;
   while (n < q_len) {
-    // Lane-local best: slots ascend with j, so a later equal weight never wins.
-    float bw = -INFINITY;
-    int bs = INT_MAX;
-#pragma unroll
-    for (int j = 0; j < kSlotRegs; ++j)
-      if (cm[j] >= 0 && (cw[j] > bw || bs == INT_MAX)) {
-        bw = cw[j];
-        bs = j * 32 + lane;
-      }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ow = __shfl_xor_sync(0xffffffffu, bw, off);
-      const int os = __shfl_xor_sync(0xffffffffu, bs, off);
-      if (os != INT_MAX && (bs == INT_MAX || ow > bw || (ow == bw && os < bs))) {
-        bw = ow;
-        bs = os;
+    // Lane-local best: a lane's slots ascend, so a later equal key never wins.
+    uint32_t bk = 0u;
+    uint32_t bs = 0xffffffffu;
+    for (int sl = lane; sl < n_slots; sl += 32) {
+      const uint32_t key = s_ck[sl];
+      if (key > bk) {
+        bk = key;
+        bs = static_cast<uint32_t>(sl);
       }
     }
-    if (bs == INT_MAX) break;  // no candidate left
-    int mine = 0;
-#pragma unroll
-    for (int j = 0; j < kSlotRegs; ++j)
-      if (j == (bs >> 5) && lane == (bs & 31)) {
-        mine = cm[j];
-        cm[j] = -1;
-      }
-    const int meta = __shfl_sync(0xffffffffu, mine, bs & 31);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
+    if (kmax == 0u) break;  // no candidate left
+    const uint32_t win = __reduce_min_sync(0xffffffffu, bk == kmax ? bs : 0xffffffffu);
+    __syncwarp();  // every lane has read the keys before the winner's is cleared
+    if (lane == 0) s_ck[win] = 0u;
+    const float bw = s_cw[win];
+    const int meta = s_cm[win];
     const int d = meta & 0xff, r = (meta >> 8) & 0xff, par = meta >> 16;
     const int node = n++;
     if (lane == 0) {
@@ -153,6 +148,7 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
       const float w = __fadd_rn(__fsub_rn(bw, s_lp[(d - 1) * Kp + r]), s_lp[(d - 1) * Kp + r + 1]);
       insert(w, d | ((r + 1) << 8) | (par << 16));
     }
+    __syncwarp();  // the new slots are visible to every lane
   }
   __syncwarp();
 

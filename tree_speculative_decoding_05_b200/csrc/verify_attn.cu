@@ -70,16 +70,23 @@ constexpr int kStageBytes = 8192;
 #ifndef DDT_VERIFY_V_STAGES
 #define DDT_VERIFY_V_STAGES 6
 #endif
+// P buffers in shared memory: the softmax of tile G writes P into buffer
+// G % kPBufs once the P V of tile G - kPBufs has read it.
+#ifndef DDT_VERIFY_P_BUFS
+#define DDT_VERIFY_P_BUFS 2
+#endif
 constexpr int kKStages = DDT_VERIFY_K_STAGES;      // each of the two K rings (even / odd tiles)
 constexpr int kVStages = DDT_VERIFY_V_STAGES;      // V ring (feeds O += P V)
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
 constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
+constexpr int kPBufs = DDT_VERIFY_P_BUFS;
+static_assert(kPBufs == 2 || kPBufs == 3, "two or three P buffers");
 constexpr int kOffQ = 0;
 constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
 constexpr int kOffVRing = kOffKRing + 2 * kKStages * kStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
-constexpr int kOffRedMax = kOffP + 2 * kPBufBytes;     // float[2][128]
+constexpr int kOffRedMax = kOffP + kPBufs * kPBufBytes;  // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
 constexpr int kMaxSortedB = 512;  // requests ordered by length (larger B: natural order)
 constexpr int kOffLen = kOffRedL + 128 * 4;            // int32[kMaxSortedB]
@@ -95,9 +102,9 @@ constexpr int kBarVEmpty = kBarVFull + kVStages;
 constexpr int kBarQ = kBarVEmpty + kVStages;
 constexpr int kBarS = kBarQ + 1;           // four S buffers: S ready
 constexpr int kBarSFree = kBarS + 4;       // four S buffers: read by both CTAs' softmax
-constexpr int kBarP = kBarSFree + 4;
-constexpr int kBarO = kBarP + 2;           // two: P V of even / odd tiles done
-constexpr int kBarQKDone = kBarO + 2;      // two: one per S issuer
+constexpr int kBarP = kBarSFree + 4;      // kPBufs: P of tile G written (G % kPBufs)
+constexpr int kBarO = kBarP + kPBufs;      // four: P V of tile G done (G % 4)
+constexpr int kBarQKDone = kBarO + 4;      // two: one per S issuer
 constexpr int kBarPVDone = kBarQKDone + 2;
 constexpr int kBarQFree = kBarPVDone + 1;  // both S issuers are done with this item's Q
 constexpr int kBarOFree = kBarQFree + 1;   // both CTAs' epilogues have read O
@@ -250,9 +257,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_init(bar(kBarS + s), 1);
       mbar_init(bar(kBarSFree + s), 2);  // one arrival per CTA of the pair
     }
-    for (int s = 0; s < 2; ++s) mbar_init(bar(kBarP + s), 2);  // one arrival per CTA
-    mbar_init(bar(kBarO + 0), 1);
-    mbar_init(bar(kBarO + 1), 1);
+    for (int s = 0; s < kPBufs; ++s) mbar_init(bar(kBarP + s), 2);  // one arrival per CTA
+    for (int s = 0; s < 4; ++s) mbar_init(bar(kBarO + s), 1);
     mbar_init(bar(kBarQKDone + 0), 1);
     mbar_init(bar(kBarQKDone + 1), 1);
     mbar_init(bar(kBarPVDone), 1);
@@ -444,8 +450,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           tc_fence_after_sync();
         }
         for (int jj = 0; jj < it.ntile; ++jj, ++G) {
-          const int pb = static_cast<int>(G & 1);
-          mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((G >> 1) & 1), abort_flag);
+          const int pb = static_cast<int>(G % kPBufs);
+          mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((G / kPBufs) & 1), abort_flag);
           tc_fence_after_sync();
           for (int kb = 0; kb < 4; ++kb) {
             for (int nh = 0; nh < 2; ++nh) {
@@ -462,7 +468,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
               r.advance(kVStages);
             }
           }
-          mma_commit<2>(bar(kBarO + static_cast<int>(G & 1)), 0x3);
+          mma_commit<2>(bar(kBarO + static_cast<int>(G & 3)), 0x3);
         }
         ++iter;
       }
@@ -481,13 +487,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     const uint32_t s_free_leader0 = map_to_rank(bar(kBarSFree), 0);
     const uint32_t o_free_leader = map_to_rank(bar(kBarOFree), 0);
     // P V completions are confirmed strictly in tile order (o_next = the next
-    // tile to confirm) on two barriers alternating by tile parity, so a wait
-    // never sees a barrier more than one phase ahead of it.
+    // tile to confirm) on four barriers taken by tile % 4.  The softmax waits at
+    // most for tile G - kPBufs while P V can have finished at most tile G - 1,
+    // so a wait never sees a barrier more than one phase ahead of it.
     int64_t o_next = 0;
     auto wait_o_through = [&](int64_t last) {
       bool waited = false;
       while (o_next <= last) {
-        mbar_wait(bar(kBarO + static_cast<int>(o_next & 1)), static_cast<uint32_t>((o_next >> 1) & 1),
+        mbar_wait(bar(kBarO + static_cast<int>(o_next & 3)), static_cast<uint32_t>((o_next >> 2) & 1),
                   abort_flag);
         ++o_next;
         waited = true;
@@ -516,7 +523,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       float m_use = 0.f;
       for (int jj = 0; jj < ntile; ++jj, ++G) {
         const int tile = t0 + jj;
-        const int sb = static_cast<int>(G & 1);              // P buffer, exchange slot
+        const int sb = static_cast<int>(G & 1);              // max-exchange slot
+        const int pbuf = static_cast<int>(G % kPBufs);       // P buffer
         const int sbuf = static_cast<int>(G & (kNumS - 1));  // S buffer
         mbar_wait(bar(kBarS + sbuf), static_cast<uint32_t>((G >> 2) & 1), abort_flag);
         tc_fence_after_sync();
@@ -580,10 +588,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           pk[c] = pack_bf16x2(e0, e1);
           l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
         }
-        // The P buffer of this tile was last read by the P V of tile G-2.
-        wait_o_through(G - 2);
+        // The P buffer of this tile was last read by the P V of tile G - kPBufs.
+        wait_o_through(G - kPBufs);
         // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
-        uint8_t* prow = base + kOffP + sb * kPBufBytes + hf * kStageBytes + m * 128;
+        uint8_t* prow = base + kOffP + pbuf * kPBufBytes + hf * kStageBytes + m * 128;
 #pragma unroll
         for (int c16 = 0; c16 < 8; ++c16) {
           uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
@@ -610,7 +618,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_barrier_sync(2, kSoftmaxThreads);
-        if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * sb);
+        if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * pbuf);
       }
       // ----------------------------------------------------------- epilogue
       wait_o_through(G - 1);
