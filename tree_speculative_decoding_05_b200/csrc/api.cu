@@ -61,6 +61,41 @@ cudaError_t ensure_smem_limit(const void* func, int bytes, int slot) {
   return cudaSuccess;
 }
 
+// Split plan of the verify kernel (host side).
+int verify_num_splits(const ddt_attn_args& a, int sm_count) {
+  if (a.num_splits > 0) return a.num_splits;
+  const int n_pairs = (a.q_len + 1) / 2;
+  const int64_t items = static_cast<int64_t>(a.B) * n_pairs;
+  const int64_t pairs_avail = sm_count / 2 > 0 ? sm_count / 2 : 1;
+  const int max_tiles = (a.max_prefix + a.q_len + 127) / 128;
+  // Estimated time in KV-tile units: waves of work items x (tiles per item + a
+  // fixed cost per item: its Q load, pipeline fill and epilogue), plus, with
+  // several splits, writing and merging the partials.  The two constants (4 tiles
+  // per item, 0.75 tile per split) are fitted to measured split sweeps (one
+  // request with a 32768-row prefix: 4 splits 149 us, 8: 162, 13: 169, 16: 203).
+  auto cost = [&](int s) {
+    const int64_t waves = (items * s + pairs_avail - 1) / pairs_avail;
+    const int per = (max_tiles + s - 1) / s;
+    return static_cast<double>(waves) * (per + 4.0) + (s > 1 ? 0.75 * s : 0.0);
+  };
+  int best = 1;
+  double best_cost = cost(1);
+  for (int s = 2; s <= 32 && s <= max_tiles; ++s) {
+    const double c = cost(s);
+    if (c < best_cost) {
+      best = s;
+      best_cost = c;
+    }
+  }
+  return best;
+}
+
+size_t verify_workspace_bytes(const ddt_attn_args& a, int num_splits) {
+  if (num_splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(a.B) * a.q_len * 64;
+  return static_cast<size_t>(num_splits) * rows * (512 + 1) * sizeof(float);
+}
+
 }  // namespace ddt
 
 using namespace ddt;

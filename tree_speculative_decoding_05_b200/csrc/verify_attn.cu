@@ -796,39 +796,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
 
 }  // namespace
 
-int verify_num_splits(const ddt_attn_args& a, int sm_count) {
-  if (a.num_splits > 0) return a.num_splits;
-  const int n_pairs = (a.q_len + 1) / 2;
-  const int64_t items = static_cast<int64_t>(a.B) * n_pairs;
-  const int pairs_avail = sm_count / 2 > 0 ? sm_count / 2 : 1;
-  const int max_tiles = (a.max_prefix + a.q_len + 127) / 128;
-  // Score = wave efficiency x share of a work item spent on KV tiles (each item
-  // also pays about 1.5 tiles of fixed cost: set-up, Q load, pipeline fill).
-  auto score = [&](int s) {
-    const int64_t n = items * s;
-    const int64_t waves = (n + pairs_avail - 1) / pairs_avail;
-    const double eff = static_cast<double>(n) / static_cast<double>(waves * pairs_avail);
-    const int per = (max_tiles + s - 1) / s;
-    return eff * per / (per + 1.5);
-  };
-  int best = 1;
-  double best_score = score(1);
-  for (int s = 2; s <= 32 && s <= max_tiles; ++s) {
-    const double sc = score(s);
-    if (sc > best_score * 1.02) {
-      best = s;
-      best_score = sc;
-    }
-  }
-  return best;
-}
-
-size_t verify_workspace_bytes(const ddt_attn_args& a, int num_splits) {
-  if (num_splits <= 1) return 0;
-  const size_t rows = static_cast<size_t>(a.B) * a.q_len * 64;
-  return static_cast<size_t>(num_splits) * rows * (512 + 1) * sizeof(float);
-}
-
 namespace {
 
 // One launch of the verify kernel over key range `kv_mode` (see VerifyParams).
