@@ -67,16 +67,17 @@ int verify_num_splits(const ddt_attn_args& a, int sm_count) {
   const int n_pairs = (a.q_len + 1) / 2;
   const int64_t items = static_cast<int64_t>(a.B) * n_pairs;
   const int64_t pairs_avail = sm_count / 2 > 0 ? sm_count / 2 : 1;
-  const int max_tiles = (a.max_prefix + a.q_len + 127) / 128;
-  // Estimated time in KV-tile units: waves of work items x (tiles per item + a
-  // fixed cost per item: its Q load, pipeline fill and epilogue), plus, with
-  // several splits, writing and merging the partials.  The two constants (4 tiles
-  // per item, 0.75 tile per split) are fitted to measured split sweeps (one
+  const int max_tiles = (a.max_prefix + a.q_len + kVerifyTileKeys - 1) / kVerifyTileKeys;
+  const double rows128 = kVerifyTileKeys / 128.0;  // a tile's work in 128-row units
+  // Estimated time in units of one 128-row tile: waves of work items x (tiles per
+  // item + a fixed cost per item: its Q load, pipeline fill and epilogue), plus,
+  // with several splits, writing and merging the partials.  The two constants (4
+  // units per item, 0.75 per split) are fitted to measured split sweeps (one
   // request with a 32768-row prefix: 4 splits 149 us, 8: 162, 13: 169, 16: 203).
   auto cost = [&](int s) {
     const int64_t waves = (items * s + pairs_avail - 1) / pairs_avail;
     const int per = (max_tiles + s - 1) / s;
-    return static_cast<double>(waves) * (per + 4.0) + (s > 1 ? 0.75 * s : 0.0);
+    return static_cast<double>(waves) * (per * rows128 + 4.0) + (s > 1 ? 0.75 * s : 0.0);
   };
   int best = 1;
   double best_cost = cost(1);

@@ -9,7 +9,15 @@
 
 #include "ddt.h"
 
+// Rows of the latent cache per KV tile of the verify kernel (128, or 256 for the
+// wide-tile build); the host-side split plan counts tiles of this size.
+#ifndef DDT_VERIFY_TILE_KEYS
+#define DDT_VERIFY_TILE_KEYS 128
+#endif
+
 namespace ddt {
+
+constexpr int kVerifyTileKeys = DDT_VERIFY_TILE_KEYS;
 
 cudaError_t launch_tree_build(const float* lp, const int32_t* tok, const int32_t* root_token,
                               int B, int D, int K, int q_len, int32_t* parents,

@@ -63,9 +63,15 @@ namespace ddt {
 namespace va {
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kStageBytes = 8192;
+constexpr int kStageBytes = 8192;                  // Q chunk, V stage, P chunk: 64 x 128 B
+// KV tile: kTK cache rows per tile; each CTA of the pair stages kKH of them for
+// S = Q K^T (the pair's MMA has N = kTK).
+constexpr int kTK = DDT_VERIFY_TILE_KEYS;
+static_assert(kTK == 128 || kTK == 256, "KV tiles of 128 or 256 rows");
+constexpr int kKH = kTK / 2;
+constexpr int kKStageBytes = kKH * 128;            // K stage: kKH keys x 64 dims
 #ifndef DDT_VERIFY_K_STAGES
-#define DDT_VERIFY_K_STAGES 4
+#define DDT_VERIFY_K_STAGES (DDT_VERIFY_TILE_KEYS == 128 ? 4 : 2)
 #endif
 #ifndef DDT_VERIFY_V_STAGES
 #define DDT_VERIFY_V_STAGES 6
@@ -73,18 +79,19 @@ constexpr int kStageBytes = 8192;
 // P buffers in shared memory: the softmax of tile G writes P into buffer
 // G % kPBufs once the P V of tile G - kPBufs has read it.
 #ifndef DDT_VERIFY_P_BUFS
-#define DDT_VERIFY_P_BUFS 2
+#define DDT_VERIFY_P_BUFS (DDT_VERIFY_TILE_KEYS == 128 ? 2 : 1)
 #endif
 constexpr int kKStages = DDT_VERIFY_K_STAGES;      // each of the two K rings (even / odd tiles)
 constexpr int kVStages = DDT_VERIFY_V_STAGES;      // V ring (feeds O += P V)
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
-constexpr int kPBufBytes = 2 * kStageBytes;        // 64 rows x 128 keys bf16
+constexpr int kPBufBytes = kTK * 128;              // 64 rows x kTK keys bf16
 constexpr int kPBufs = DDT_VERIFY_P_BUFS;
-static_assert(kPBufs == 2 || kPBufs == 3, "two or three P buffers");
+static_assert(kPBufs >= 1 && kPBufs <= 3, "one to three P buffers");
+constexpr int kVBlocks = kTK / 32;                 // 32-key V blocks per tile
 constexpr int kOffQ = 0;
 constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
-constexpr int kOffVRing = kOffKRing + 2 * kKStages * kStageBytes;
+constexpr int kOffVRing = kOffKRing + 2 * kKStages * kKStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffRedMax = kOffP + kPBufs * kPBufBytes;  // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
@@ -116,10 +123,13 @@ constexpr int kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr int kTmemCols = 512;
-constexpr int kNumS = 4;     // S buffers at columns 0, 64, 128, 192
+constexpr int kSCols = kTK / 2;          // TMEM columns of one S buffer
+constexpr int kNumS = 256 / kSCols;      // S buffers in columns [0, 256): 4 or 2
+constexpr int kLogNumS = kNumS == 4 ? 2 : 1;
+constexpr int kSChunks = kKH / 64;       // 64-key chunks of S per softmax thread
 constexpr int kTmemS = 0;
 constexpr int kTmemO = 256;  // O halves at columns 256 and 384
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kTK, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, false, true);
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -145,7 +155,7 @@ struct VerifyParams {
 
 // KV tile range [t0, t1) of split `split` for a cache of T rows.
 __host__ __device__ inline void split_range(int T, int num_splits, int split, int& t0, int& t1) {
-  const int n_tiles = (T + 127) / 128;
+  const int n_tiles = (T + kVerifyTileKeys - 1) / kVerifyTileKeys;
   const int per = (n_tiles + num_splits - 1) / num_splits;
   t0 = split * per;
   t1 = t0 + per < n_tiles ? t0 + per : n_tiles;
@@ -175,7 +185,7 @@ __device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int w, co
   int t0 = 0, t1 = 0;
   if (!it.bad_prefix) {
     if (p.kv_mode == 2) {
-      t0 = (it.T + 127) / 128 - 1;  // the one tile ending at T holds the tree block (Q <= 128)
+      t0 = (it.T + va::kTK - 1) / va::kTK - 1;  // the one tile ending at T holds the tree block
       t1 = t0 + 1;
     } else {
       split_range(it.end, p.num_splits, it.split, t0, t1);
@@ -183,7 +193,7 @@ __device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int w, co
   }
   it.t0 = t0;
   it.ntile = t1 - t0;  // 0 for an empty split (the merge skips it)
-  it.last_tile = (it.end + 127) / 128 - 1;
+  it.last_tile = (it.end + va::kTK - 1) / va::kTK - 1;
   it.valid = !it.bad_prefix && it.ntile > 0;
   return it;
 }
@@ -191,9 +201,9 @@ __device__ __forceinline__ WorkItem decode_item(const VerifyParams& p, int w, co
 // First cache row of KV tile t.  A request's last tile is shifted to end at the
 // pass's last row (T, or P for a prefix pass), so no load ever reaches the rows
 // past it (padding that may hold anything); its overlap with the previous tile
-// is masked, and rows below 0 (fewer than 128 rows) read as zeros.
+// is masked, and rows below 0 (fewer than kTK rows) read as zeros.
 __device__ __forceinline__ int tile_start(const WorkItem& it, int t) {
-  return t == it.last_tile ? it.end - 128 : 128 * t;
+  return t == it.last_tile ? it.end - va::kTK : va::kTK * t;
 }
 
 // The k-th work index of a cluster: rounds of n_clusters indices, alternating
@@ -321,9 +331,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     // complete bytes on them.
     if (lane == 0) {
       const int g = warp == 4 ? 0 : 1;
-      const int key_half = static_cast<int>(rank) * 64;
+      const int key_half = static_cast<int>(rank) * kKH;
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
-      const uint32_t ring = sKRing + g * kKStages * kStageBytes;
+      const uint32_t ring = sKRing + g * kKStages * kKStageBytes;
       const uint32_t qbar = map_to_rank(bar(kBarQ), 0);
       Ring r;
       int iter = 0;
@@ -347,9 +357,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           const int key0 = tile_start(it, it.t0 + jj) + key_half;
           for (int c = 0; c < kQChunks; ++c) {
             mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
-            if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kStageBytes);
+            if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kKStageBytes);
             const uint32_t fb = map_to_rank(bar(full0 + r.stage), 0);
-            const uint32_t dst = ring + r.stage * kStageBytes;
+            const uint32_t dst = ring + r.stage * kKStageBytes;
             if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, it.b);
             else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, it.b);
             r.advance(kKStages);
@@ -369,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         const WorkItem it = decode_item(p, item, order);
         if (!it.valid) continue;
         for (int jj = 0; jj < it.ntile; ++jj) {
-          for (int kb = 0; kb < 4; ++kb) {
+          for (int kb = 0; kb < kVBlocks; ++kb) {
             const int key0 = tile_start(it, it.t0 + jj) + 32 * kb;
             for (int nh = 0; nh < 2; ++nh) {
               mbar_wait(bar(kBarVEmpty + r.stage), r.phase ^ 1u, abort_flag);
@@ -393,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     if (leader && lane == 0) {
       const int g = warp == 5 ? 0 : 1;
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
-      const uint32_t ring = sKRing + g * kKStages * kStageBytes;
+      const uint32_t ring = sKRing + g * kKStages * kKStageBytes;
       Ring r;
       int iter = 0;
       int64_t G = 0;
@@ -408,14 +418,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           const int sbuf = static_cast<int>(G & (kNumS - 1));
           if (G >= kNumS) {
             // S buffer sbuf is free once both CTAs' softmax has read tile G-4.
-            mbar_wait(bar(kBarSFree + sbuf), static_cast<uint32_t>(((G >> 2) - 1) & 1), abort_flag);
+            mbar_wait(bar(kBarSFree + sbuf), static_cast<uint32_t>(((G >> kLogNumS) - 1) & 1),
+                      abort_flag);
             tc_fence_after_sync();
           }
-          const uint32_t d = tmem + kTmemS + 64u * static_cast<uint32_t>(sbuf);
+          const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(kSCols * sbuf);
           for (int c = 0; c < kQChunks; ++c) {
             mbar_wait(bar(full0 + r.stage), r.phase, abort_flag);
             const uint32_t a0 = sQ + c * kStageBytes;
-            const uint32_t b0 = ring + r.stage * kStageBytes;
+            const uint32_t b0 = ring + r.stage * kKStageBytes;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
@@ -453,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           const int pb = static_cast<int>(G % kPBufs);
           mbar_wait(bar(kBarP + pb), static_cast<uint32_t>((G / kPBufs) & 1), abort_flag);
           tc_fence_after_sync();
-          for (int kb = 0; kb < 4; ++kb) {
+          for (int kb = 0; kb < kVBlocks; ++kb) {
             for (int nh = 0; nh < 2; ++nh) {
               mbar_wait(bar(kBarVFull + r.stage), r.phase, abort_flag);
               const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
@@ -526,46 +537,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         const int sb = static_cast<int>(G & 1);              // max-exchange slot
         const int pbuf = static_cast<int>(G % kPBufs);       // P buffer
         const int sbuf = static_cast<int>(G & (kNumS - 1));  // S buffer
-        mbar_wait(bar(kBarS + sbuf), static_cast<uint32_t>((G >> 2) & 1), abort_flag);
+        mbar_wait(bar(kBarS + sbuf), static_cast<uint32_t>((G >> kLogNumS) & 1), abort_flag);
         tc_fence_after_sync();
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_addr + kTmemS + 64u * sbuf, r0);
-        tmem_ld32(tmem + lane_addr + kTmemS + 64u * sbuf + 32u, r1);
-        tmem_wait_ld();
-        tc_fence_before_sync();
-        float x[64];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(r0[c]) * p.scale_log2;
-          x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
-        }
-        const int key0 = tile_start(it, tile) + hf * 64;
+        // This thread's keys of the tile: [kbase, kbase + kKH), in chunks of 64.
+        const int kbase = tile_start(it, tile) + hf * kKH;
         // Keys below lo belong to the previous tile (a tree-block pass has none).
         // Prefix rows are visible to every node, except in a tree-block pass,
         // whose one tile may also reach prefix rows and rows below 0.
         const bool tree_pass = p.kv_mode == 2;
-        const int lo = tree_pass ? INT_MIN : tile * 128;
-        if (tree_pass || key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
+        const int lo = tree_pass ? INT_MIN : tile * kTK;
+        // Scaled, masked scores of 64-key chunk sc (log2 units).
+        auto load_chunk = [&](int sc, float (&x)[64]) {
+          uint32_t r0[32], r1[32];
+          const uint32_t col = tmem + lane_addr + kTmemS + static_cast<uint32_t>(kSCols * sbuf + 64 * sc);
+          tmem_ld32(col, r0);
+          tmem_ld32(col + 32u, r1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int key = key0 + c;
-            bool vis = !tree_pass && key < P;
-            if (!vis && key >= P && key < T) {
-              const int a = key - P;
-              const uint64_t w = a < 64 ? mw0 : mw1;
-              vis = (w >> (a & 63)) & 1ull;
-            }
-            if (key < lo) vis = false;
-            if (!vis) x[c] = -INFINITY;
+          for (int c = 0; c < 32; ++c) {
+            x[c] = __uint_as_float(r0[c]) * p.scale_log2;
+            x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
           }
-        }
+          const int key0 = kbase + 64 * sc;
+          if (tree_pass || key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const int key = key0 + c;
+              bool vis = !tree_pass && key < P;
+              if (!vis && key >= P && key < T) {
+                const int a = key - P;
+                const uint64_t w = a < 64 ? mw0 : mw1;
+                vis = (w >> (a & 63)) & 1ull;
+              }
+              if (key < lo) vis = false;
+              if (!vis) x[c] = -INFINITY;
+            }
+          }
+        };
+        float x[64];
+        load_chunk(0, x);
         float mx = x[0];
 #pragma unroll
         for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+        // Wider tiles: the other chunks' maxima now; their scores are reloaded below.
+#pragma unroll 1
+        for (int sc = 1; sc < kSChunks; ++sc) {
+          load_chunk(sc, x);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) mx = fmaxf(mx, x[c]);
+        }
+        if (kSChunks == 1) tc_fence_before_sync();
         red_max[sb * 128 + t] = mx;
         named_barrier_sync(1, kSoftmaxThreads);
         // Every thread of this CTA has read S: release the buffer.
-        if (t == 0) mbar_arrive_cluster(s_free_leader0 + 8u * sbuf);
+        if (kSChunks == 1 && t == 0) mbar_arrive_cluster(s_free_leader0 + 8u * sbuf);
         mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]);
         float factor = 1.f;
         bool rescale = false;
@@ -578,25 +603,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           rescale = true;
         }
         m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // The row sum takes the bf16-rounded weights, the values the P V product
-        // multiplies, so the normalised weights sum to one exactly.
-        uint32_t pk[32];
+#pragma unroll 1
+        for (int sc = 0; sc < kSChunks; ++sc) {
+          if (sc > 0 || kSChunks > 1) load_chunk(sc, x);
+          // The row sum takes the bf16-rounded weights, the values the P V product
+          // multiplies, so the normalised weights sum to one exactly.
+          uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = fast_exp2(x[2 * c] - m_use);
-          const float e1 = fast_exp2(x[2 * c + 1] - m_use);
-          pk[c] = pack_bf16x2(e0, e1);
-          l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
-        }
-        // The P buffer of this tile was last read by the P V of tile G - kPBufs.
-        wait_o_through(G - kPBufs);
-        // P tile: K-major, 128-byte swizzle, chunk hf holds keys [64 hf, 64 hf + 64).
-        uint8_t* prow = base + kOffP + pbuf * kPBufBytes + hf * kStageBytes + m * 128;
+          for (int c = 0; c < 32; ++c) {
+            const float e0 = fast_exp2(x[2 * c] - m_use);
+            const float e1 = fast_exp2(x[2 * c + 1] - m_use);
+            pk[c] = pack_bf16x2(e0, e1);
+            l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+          }
+          // The P buffer of this tile was last read by the P V of tile G - kPBufs.
+          if (sc == 0) wait_o_through(G - kPBufs);
+          // P tile: K-major, 128-byte swizzle, 64-key chunks of 8 KB; this thread's
+          // chunk sc holds keys [hf kKH + 64 sc, + 64) of the tile.
+          uint8_t* prow = base + kOffP + pbuf * kPBufBytes +
+                          (hf * kSChunks + sc) * kStageBytes + m * 128;
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-          *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
+          for (int c16 = 0; c16 < 8; ++c16) {
+            uint4 v = make_uint4(pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
+            *reinterpret_cast<uint4*>(prow + ((c16 ^ (m & 7)) << 4)) = v;
+          }
         }
+        if (kSChunks > 1) tc_fence_before_sync();
         if (jj > 0) {
           if (__any_sync(0xffffffffu, rescale)) {
             // O may be rescaled only once the P V of the previous tile is done
@@ -618,7 +650,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_barrier_sync(2, kSoftmaxThreads);
-        if (t == 0) mbar_arrive_cluster(p_full_leader0 + 8u * pbuf);
+        if (t == 0) {
+          if (kSChunks > 1) mbar_arrive_cluster(s_free_leader0 + 8u * sbuf);  // S read twice
+          mbar_arrive_cluster(p_full_leader0 + 8u * pbuf);
+        }
       }
       // ----------------------------------------------------------- epilogue
       wait_o_through(G - 1);
@@ -808,9 +843,9 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
   const uint64_t cap = static_cast<uint64_t>(a.capacity);
   bool ok = make_map(&m_qlat, a.q_lat, 512, rows_q, B, 512 * 2, rows_q * 512 * 2, 64) &&
             make_map(&m_qrope, a.q_rope, 64, rows_q, B, 64 * 2, rows_q * 64 * 2, 64) &&
-            make_map(&m_ckv_k, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 64) &&
+            make_map(&m_ckv_k, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, kKH) &&
             make_map(&m_ckv_v, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 32) &&
-            make_map(&m_krope, a.k_rope, 64, cap, B, a.kr_row_stride * 2, a.kr_batch_stride * 2, 64);
+            make_map(&m_krope, a.k_rope, 64, cap, B, a.kr_row_stride * 2, a.kr_batch_stride * 2, kKH);
   if (!ok) return DDT_ERR_INVALID_ARG;
   if (ensure_smem_limit(reinterpret_cast<const void*>(verify_attn_kernel), kSmemBytes, 1) !=
       cudaSuccess)
