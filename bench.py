@@ -576,6 +576,34 @@ def per_call_report(args) -> int:
     return 0
 
 
+def accept_sweep() -> int:
+    """tree_accept timed alone on random trees (depth <= 15) for streams {1, 8, 64} x
+    draft budget {8, 32} (q_len = budget + 1): 100 calls in a CUDA graph, median of 5."""
+    import torch
+
+    from tree_speculative_decoding_05_b200 import ddt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    res = {}
+    for streams in (1, 8, 64):
+        for budget in (8, 32):
+            w = inputs.make_workload("accept", 500 + streams + budget, streams, budget + 1,
+                                     [0] * streams, heads=1, d_latent=8, d_rope=8)
+            t = {k: torch.from_numpy(np.ascontiguousarray(getattr(w, k))).to(dev)
+                 for k in ("node_tokens", "target_tokens", "next_token", "next_sibling")}
+            path = torch.empty((streams, budget + 1), dtype=torch.int32, device=dev)
+            alen = torch.empty((streams,), dtype=torch.int32, device=dev)
+            fn = lambda: ddt.tree_accept(t["node_tokens"], t["target_tokens"], t["next_token"],
+                                         t["next_sibling"], path=path, accept_len=alen)
+            for _ in range(10):
+                fn()
+            res[f"streams={streams},budget={budget}"] = graph_time_us(fn, 100)
+    print(json.dumps({"tree_accept_us": res, "timing": "100 calls per CUDA graph, median of 5"}),
+          flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -592,6 +620,9 @@ def main(argv=None) -> int:
                          "warm L2 and after a 256 MB L2 flush), plus the oracle on all host "
                          "cores and on one; one JSON line per workload")
     ap.add_argument("--configs", type=str, default="0,1,2,3,4")
+    ap.add_argument("--accept-sweep", action="store_true",
+                    help="tree_accept alone over streams {1, 8, 64} x budget {8, 32} (the grid "
+                         "the pages report), graph-timed; one JSON line")
     ap.add_argument("--shard", choices=["replicas", "lpt"], default="replicas",
                     help="with several GPUs: every rank runs its own batch of the workload "
                          "(replicas, weak scaling) or the ranks split one batch by request "
@@ -607,6 +638,8 @@ def main(argv=None) -> int:
 
     if args.per_call:
         return per_call_report(args)
+    if args.accept_sweep:
+        return accept_sweep()
     if args.impl == "reference":
         if rank != 0:
             return 0

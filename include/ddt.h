@@ -351,10 +351,9 @@ DDT_API ddt_status ddt_kv_compact(void* c_kv, void* k_rope, int64_t ckv_batch_st
 /* ------------------------------------------------------------------------ */
 /* ddt_tree_accept followed by ddt_kv_compact of its path, in one launch.
  *
- * Source: [Race Conditions] "Race Conditions, Buffer Aliasing, and the
- * Architecture of a Native DDTree Inference Engine" (the compaction gather of
- * the accepted rows; fusing that gather is named there as work still to do)
- * and the walk of ddt_tree_accept.  Results are exactly those of the two calls
+ * Source: [Race Conditions] "The Cache Compaction Problem" (the gather of the
+ * accepted rows) and "The Broader Significance" (fusing that gather is deferred
+ * there to a later phase), and the walk of ddt_tree_accept.  Results are exactly those of the two calls
  * in sequence: path, accept_len, bonus_token and accept_status as
  * ddt_tree_accept writes them, then the cache rows, new_prefix_lens and
  * compact_status as ddt_kv_compact writes them for that path (which can only

@@ -4,10 +4,10 @@
  * smoke check and by the benchmark's CPU-baseline leg, never by the product
  * path.  It shares no code, header or constant with the CUDA library.
  *
- * Every floating-point step is done in double precision on inputs that are
- * bfloat16 bit patterns widened exactly.  Each function follows the written
- * definition of its step, in the order of the definition, with no blocking or
- * fusion.
+ * Attention is done in double precision on inputs that are bfloat16 bit
+ * patterns widened exactly; the tree build's weights are float32, the precision
+ * the pages fix for them.  Each function follows the written definition of its
+ * step, in the order of the definition, with no blocking or fusion.
  *
  * Sources (page title, section):
  *   [Race Conditions] "Race Conditions, Buffer Aliasing, and the Architecture of

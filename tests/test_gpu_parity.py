@@ -247,3 +247,33 @@ def test_step_configs_accept_and_compact():
         assert np.array_equal(dw.c_kv.view(torch.int16).cpu().numpy().view(np.uint16), c_ref)
         assert np.array_equal(dw.k_rope.view(torch.int16).cpu().numpy().view(np.uint16), k_ref)
         assert np.array_equal(newp.cpu().numpy(), p_ref) and np.array_equal(cst.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_verify_attn_random_shapes(seed):
+    """Seeded random shapes across the supported range: batch, q_len up to 128
+    (two mask words), prefixes from 0 to a few thousand rows, either output dtype,
+    forced or automatic split counts, fused or prefix/tail-split computation."""
+    rng = np.random.RandomState(900 + seed)
+    B = int(rng.randint(1, 5))
+    Q = int(rng.choice([1, 2, 5, 17, 33, 64, 65, 100, 128]))
+    P = rng.randint(0, 3000, size=B).astype(np.int32)
+    out_dtype = "f32" if rng.rand() < 0.5 else "bf16"
+    w = inputs.make_workload("fuzz", 900 + seed, B, Q, P, out_dtype=out_dtype, want_lse=True,
+                             row_scale_range=(0.5, 2.0) if rng.rand() < 0.5 else None)
+    dw = DeviceWorkload(w)
+    splits = int(rng.choice([0, 0, 1, 2, 3, 7]))
+    H = 64
+    rows = sample_rows(B, Q, H, 1024, seed=seed, must=np.arange(B * Q * H - 64, B * Q * H))
+    what = f"B={B} Q={Q} P={P.tolist()} {out_dtype} splits={splits}"
+    _check_attention(dw, rows=rows, num_splits=splits, what=what)
+    mask, _, _ = ddt.build_mask(dw.parents)
+    od = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    out, lse = ddt.verify_attn(dw.q_lat, dw.q_rope, dw.c_kv, dw.k_rope, dw.prefix, mask,
+                               w.softmax_scale, max_prefix=int(P.max()), out_dtype=od,
+                               want_lse=True, num_splits=splits, split_tail=True)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
+                                    w.parents, w.softmax_scale, rows)
+    compare_attention(rows_of(out, rows), o_ref, what + " split")
+    assert np.abs(lse.reshape(-1).cpu().numpy()[rows] - l_ref).max() <= LSE_MAX_ABS, what

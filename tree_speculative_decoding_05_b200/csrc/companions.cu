@@ -231,9 +231,9 @@ __global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Accept fused with compaction.  [Race Conditions] "Race Conditions, Buffer
-// Aliasing, ..." closes with the compaction gather as a separate step and names
-// fusing it as later work.  Here one CTA per request walks the tree (thread 0,
+// Accept fused with compaction.  [Race Conditions] "The Broader Significance"
+// defers fusing the compaction gather to a later phase, keeping it a separate
+// step.  Here one CTA per request walks the tree (thread 0,
 // the same walk as tree_accept_kernel) and then moves the accepted rows (all
 // threads, the same staging as kv_compact_kernel), so the path never leaves the
 // chip and one launch replaces two.  The walk always yields 1 <= alen <= q_len
