@@ -27,6 +27,11 @@
 //   * TMEM per CTA: four S buffers (4 x 64 cols) + O (256 cols) = all 512
 //     columns; four S buffers let S = Q K^T run up to three tiles ahead of the
 //     softmax.
+//   * Built with DDT_VERIFY_TILE_KEYS=256 the tiles hold 256 keys: S = Q K^T
+//     runs at N = 256 into two S buffers of 128 columns, each softmax thread
+//     takes its 128 keys in two 64-key chunks, and P is 32 KB per buffer.  That
+//     build is correct but slower (its shared memory leaves thinner rings), so
+//     128-key tiles are the default.
 //   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
 //     half of one query row); warps 4 and 8 TMA producers of the K rings of
 //     even and odd tiles, warp 6 the producer of the V ring; warps 5 and 9
