@@ -277,3 +277,14 @@ def test_verify_attn_random_shapes(seed):
                                     w.parents, w.softmax_scale, rows)
     compare_attention(rows_of(out, rows), o_ref, what + " split")
     assert np.abs(lse.reshape(-1).cpu().numpy()[rows] - l_ref).max() <= LSE_MAX_ABS, what
+
+
+def test_verify_attn_more_requests_than_the_length_ranking_holds():
+    """Past 512 requests the kernel keeps the natural request order instead of
+    ranking by length: 600 short ragged requests, sampled rows of every tenth."""
+    B, Q = 600, 3
+    P = inputs.ragged_prefixes(77, B, 0, 300)
+    w = inputs.make_workload("many", 77, B, Q, P, heads=64, out_dtype="bf16")
+    H = 64
+    rows = np.concatenate([np.arange(b * Q * H, (b + 1) * Q * H, 7) for b in range(0, B, 10)])
+    _check_attention(DeviceWorkload(w), rows=rows.astype(np.int64), what="600 requests")
