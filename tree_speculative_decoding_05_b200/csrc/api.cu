@@ -3,6 +3,7 @@
 // device memory or synchronises the host.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -32,16 +33,16 @@ bool cache_strides_ok(int B, int capacity, int64_t ckv_bs, int64_t ckv_rs, int64
 }  // namespace
 
 int device_sm_count() {
-  static int counts[kMaxDevices] = {0};
+  static std::atomic<int> counts[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (counts[dev] == 0) {
-    int n = 0;
+  int n = counts[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    counts[dev] = n;
+    counts[dev].store(n, std::memory_order_relaxed);
   }
-  return counts[dev];
+  return n;
 }
 
 cudaError_t ensure_smem_limit(const void* func, int bytes, int slot) {
