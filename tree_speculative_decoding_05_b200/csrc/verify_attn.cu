@@ -66,7 +66,16 @@ __device__ unsigned int ddt_fault_word = 0;  // bit set, see ddt_fault_flags
 namespace ddt {
 
 namespace va {
-constexpr int kThreads = 320;
+// S = Q K^T issuers: tile G goes to issuer G % kQKIss, each with its own K ring
+// and its own K producer warp.
+#ifndef DDT_VERIFY_QK_ISSUERS
+#define DDT_VERIFY_QK_ISSUERS 2
+#endif
+constexpr int kQKIss = DDT_VERIFY_QK_ISSUERS;
+static_assert(kQKIss == 2 || kQKIss == 3, "two or three S issuers");
+// Warps 0-3 softmax; 4 K producer 0 (and Q), 5 S issuer 0, 6 V producer, 7 P V
+// issuer, 8 K producer 1, 9 S issuer 1, 10 K producer 2, 11 S issuer 2.
+constexpr int kThreads = 32 * (6 + 2 * kQKIss);
 constexpr int kSoftmaxThreads = 128;
 constexpr int kStageBytes = 8192;                  // Q chunk, V stage, P chunk: 64 x 128 B
 // KV tile: kTK cache rows per tile; each CTA of the pair stages kKH of them for
@@ -96,7 +105,7 @@ static_assert(kPBufs >= 1 && kPBufs <= 3, "one to three P buffers");
 constexpr int kVBlocks = kTK / 32;                 // 32-key V blocks per tile
 constexpr int kOffQ = 0;
 constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
-constexpr int kOffVRing = kOffKRing + 2 * kKStages * kKStageBytes;
+constexpr int kOffVRing = kOffKRing + kQKIss * kKStages * kKStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffRedMax = kOffP + kPBufs * kPBufBytes;  // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
@@ -108,17 +117,17 @@ constexpr int kOffBar = kOffOrder + kMaxSortedB * 4;
 // full/empty, q_full, s_full[2], p_full[2], o_done, and one "all issued MMAs
 // done" barrier per issuing thread (two S issuers, one O issuer).
 constexpr int kBarKFull = 0;
-constexpr int kBarKEmpty = kBarKFull + 2 * kKStages;
-constexpr int kBarVFull = kBarKEmpty + 2 * kKStages;
+constexpr int kBarKEmpty = kBarKFull + kQKIss * kKStages;
+constexpr int kBarVFull = kBarKEmpty + kQKIss * kKStages;
 constexpr int kBarVEmpty = kBarVFull + kVStages;
 constexpr int kBarQ = kBarVEmpty + kVStages;
 constexpr int kBarS = kBarQ + 1;           // four S buffers: S ready
 constexpr int kBarSFree = kBarS + 4;       // four S buffers: read by both CTAs' softmax
 constexpr int kBarP = kBarSFree + 4;      // kPBufs: P of tile G written (G % kPBufs)
 constexpr int kBarO = kBarP + kPBufs;      // four: P V of tile G done (G % 4)
-constexpr int kBarQKDone = kBarO + 4;      // two: one per S issuer
-constexpr int kBarPVDone = kBarQKDone + 2;
-constexpr int kBarQFree = kBarPVDone + 1;  // both S issuers are done with this item's Q
+constexpr int kBarQKDone = kBarO + 4;      // one per S issuer
+constexpr int kBarPVDone = kBarQKDone + kQKIss;
+constexpr int kBarQFree = kBarPVDone + 1;  // every S issuer is done with this item's Q
 constexpr int kBarOFree = kBarQFree + 1;   // both CTAs' epilogues have read O
 constexpr int kNumBars = kBarOFree + 1;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
@@ -259,7 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   if (threadIdx.x == 0) {
     // Stage and Q barriers: one arrival (the even CTA's producer, expecting the
     // bytes of both CTAs); the odd CTA's loads only add completed bytes.
-    for (int s = 0; s < 2 * kKStages; ++s) {
+    for (int s = 0; s < kQKIss * kKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);  // the issuing thread's commit
     }
@@ -274,10 +283,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     }
     for (int s = 0; s < kPBufs; ++s) mbar_init(bar(kBarP + s), 2);  // one arrival per CTA
     for (int s = 0; s < 4; ++s) mbar_init(bar(kBarO + s), 1);
-    mbar_init(bar(kBarQKDone + 0), 1);
-    mbar_init(bar(kBarQKDone + 1), 1);
+    for (int g = 0; g < kQKIss; ++g) mbar_init(bar(kBarQKDone + g), 1);
     mbar_init(bar(kBarPVDone), 1);
-    mbar_init(bar(kBarQFree), 2);  // a commit of each S issuer
+    mbar_init(bar(kBarQFree), kQKIss);  // a commit of each S issuer
     mbar_init(bar(kBarOFree), 2);  // one arrival per CTA of the pair
     *abort_flag = 0;
     fence_mbar_init_cluster();
@@ -328,14 +336,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   };
   const bool leader = rank == 0;
 
-  if (warp == 4 || warp == 8) {
+  // K producer g: warp 4, 8, 10; S issuer g: the next warp (5, 9, 11).
+  const int qk_g = warp == 4 || warp == 5 ? 0 : warp == 8 || warp == 9 ? 1
+                   : warp == 10 || warp == 11 ? 2 : -1;
+  const bool k_producer = qk_g >= 0 && (warp & 1) == 0;
+  const bool s_issuer = qk_g >= 0 && (warp & 1) == 1;
+  if (k_producer) {
     // ---------------------------------------------- TMA: Q and the K rings
-    // Lane 0 issues; warp 4 loads Q and the K stages of even tiles, warp 8 those
-    // of odd tiles (by the tile counter G).  Only the even CTA arrives on the
+    // Lane 0 issues; producer g loads the K stages of tiles G with G % kQKIss == g
+    // (by the tile counter G), and producer 0 also loads Q.  Only the even CTA arrives on the
     // stage barriers (with the byte count of both CTAs); both CTAs' loads
     // complete bytes on them.
     if (lane == 0) {
-      const int g = warp == 4 ? 0 : 1;
+      const int g = qk_g;
       const int key_half = static_cast<int>(rank) * kKH;
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
       const uint32_t ring = sKRing + g * kKStages * kKStageBytes;
@@ -358,7 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           tma_load_3d_pair(sQ + 8 * kStageBytes, &tm_qrope, qbar, 0, node * 64, it.b);
         }
         for (int jj = 0; jj < it.ntile; ++jj, ++G) {
-          if (static_cast<int>(G & 1) != g) continue;
+          if (static_cast<int>(G % kQKIss) != g) continue;
           const int key0 = tile_start(it, it.t0 + jj) + key_half;
           for (int c = 0; c < kQChunks; ++c) {
             mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
@@ -401,12 +414,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5 || warp == 9) {
+  } else if (s_issuer) {
     // -------------------------------------------------------- MMA: S = Q K^T
-    // Warp 5 issues even tiles (by G), warp 9 odd tiles; tile G goes to S
-    // buffer G % 4.
+    // Issuer g takes tiles G with G % kQKIss == g; tile G goes to S buffer
+    // G % kNumS.
     if (leader && lane == 0) {
-      const int g = warp == 5 ? 0 : 1;
+      const int g = qk_g;
       const int full0 = kBarKFull + g * kKStages, empty0 = kBarKEmpty + g * kKStages;
       const uint32_t ring = sKRing + g * kKStages * kKStageBytes;
       Ring r;
@@ -419,7 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         if (!it.valid) continue;
         mbar_wait(bar(kBarQ), static_cast<uint32_t>(iter & 1), abort_flag);
         for (int jj = 0; jj < it.ntile; ++jj, ++G) {
-          if (static_cast<int>(G & 1) != g) continue;
+          if (static_cast<int>(G % kQKIss) != g) continue;
           const int sbuf = static_cast<int>(G & (kNumS - 1));
           if (G >= kNumS) {
             // S buffer sbuf is free once both CTAs' softmax has read tile G-4.
