@@ -884,6 +884,9 @@ def main(argv=None) -> int:
             "calls_us": {"build_mask": mask_ms_max * 1e3, "verify_attn": verify_ms_max * 1e3,
                          "tree_accept": accept_ms_max * 1e3, "kv_compact": compact_ms_max * 1e3},
             "kv_compact_gbs": compact_bytes / (compact_ms_max * 1e-3) / 1e9,
+            # each request's cache rows (prefix + tree block, 1152 B each) once per call
+            "kv_stream_gbs": float((w.prefix_lens.astype(np.float64) + Q).sum()) * (DL + DR) * 2
+                             / (verify_ms_max * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peak_src} {'sustained' if use_sustained else 'burst'} bf16",
