@@ -274,33 +274,38 @@ def oracle_sample_throughput(w, target_seconds: float, seed: int = 0, max_rows: 
 
 
 def run_reference(args, w):
-    """--impl reference: the CPU oracle as it stands, each step a bounded sample
-    (query rows of the attention, plus the mask/accept/compaction of the batch)."""
+    """--impl reference: the CPU oracle as it stands.  Each step is the whole path
+    (mask, every query row of the attention, accept, compaction) for one request
+    of the batch, requests taken in turn: a bounded sample with the same mix of
+    work as the GPU step."""
     import oracle
-    rows_per_step = max(32, oracle.threads() * 8)
-    total = w.B * w.q_len * H
-    rng = np.random.RandomState(1)
+    B = w.B
+    subs = {}
 
-    def step():
-        rows = np.sort(rng.choice(total, size=rows_per_step, replace=False)).astype(np.int64)
-        oracle.build_mask(w.parents)
-        oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens, w.parents,
-                         w.softmax_scale, rows)
-        path, alen, _, _ = oracle.tree_accept(w.node_tokens, w.target_tokens, w.next_token,
-                                              w.next_sibling)
-        oracle.kv_compact(w.c_kv, w.k_rope, w.prefix_lens, path, alen)
-        return flops_rows(w.prefix_lens, w.parents, rows)
+    def step(k):
+        b = k % B
+        if b not in subs:
+            subs[b] = inputs.subset(w, [b])
+        x = subs[b]
+        rows = np.arange(x.q_len * H, dtype=np.int64)
+        oracle.build_mask(x.parents)
+        oracle.attn_rows(x.q_lat, x.q_rope, x.c_kv, x.k_rope, x.prefix_lens, x.parents,
+                         x.softmax_scale, rows)
+        path, alen, _, _ = oracle.tree_accept(x.node_tokens, x.target_tokens, x.next_token,
+                                              x.next_sibling)
+        oracle.kv_compact(x.c_kv, x.k_rope, x.prefix_lens, path, alen)
+        return verify_flops(x.prefix_lens, x.parents)
 
-    for _ in range(args.warmup):
-        step()
+    for k in range(args.warmup):
+        step(k)
     t0 = time.perf_counter()
     flops = 0.0
-    for _ in range(args.steps):
-        flops += step()
+    for k in range(args.steps):
+        flops += step(args.warmup + k)
     secs = time.perf_counter() - t0
     value = flops / secs / 1e12
-    sample = (f"{rows_per_step} random query rows of the attention per step "
-              f"(of {total}) + mask, accept and compaction of the full batch")
+    sample = (f"per step one request of the {B}-request batch, in turn: its mask, all "
+              f"{w.q_len * H} query rows of its attention, its accept walk and compaction")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
