@@ -459,6 +459,16 @@ DDT_API const char* ddt_status_str(ddt_status status);
 #define DDT_FAULT_WAIT_TIMEOUT 1u
 DDT_API ddt_status ddt_fault_flags(uint32_t* flags, int32_t reset);
 
+/* Self-test of the kernels' bounded waits (no counterpart on the pages; the
+ * library's own failure detection).  Launches one thread that waits, for at most
+ * timeout_us microseconds, on a barrier that nothing will ever complete.  The
+ * wait gives up as every wait in the library does on a stalled barrier: it sets
+ * DDT_FAULT_WAIT_TIMEOUT in the fault word (read with ddt_fault_flags), writes 1
+ * to *gave_up (device int32, or NULL) and returns, leaving the context usable.
+ * timeout_us must be in [1, 1000000], else DDT_ERR_INVALID_ARG. */
+DDT_API ddt_status ddt_selftest_bounded_wait(uint32_t timeout_us, int32_t* gave_up,
+                                     ddt_stream_t stream);
+
 /* Library version string (static storage). */
 DDT_API const char* ddt_version(void);
 

@@ -926,6 +926,34 @@ ddt_status launch_verify_attn_split_tail(const ddt_attn_args& a, int prefix_spli
 
 }  // namespace ddt
 
+namespace ddt {
+// Self-test of the bounded wait: one thread waits, with a short limit, for the
+// first phase of a barrier that nothing arrives at.  The wait must give up,
+// record the fault bit and return; *gave_up is set to 1 when it did.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar_storage), 1);
+    abort_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool completed = mbar_wait(smem_u32(&bar_storage), 0u, &abort_flag, timeout_ns);
+    if (gave_up) *gave_up = completed ? 0 : 1;
+  }
+}
+}  // namespace ddt
+
+extern "C" ddt_status ddt_selftest_bounded_wait(uint32_t timeout_us, int32_t* gave_up,
+                                                ddt_stream_t stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u) return DDT_ERR_INVALID_ARG;
+  ddt::wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull, gave_up);
+  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+}
+
 // Diagnostic read of the library's device fault word (synchronises the device).
 extern "C" ddt_status ddt_fault_flags(uint32_t* flags, int32_t reset) {
   if (!flags) return DDT_ERR_INVALID_ARG;

@@ -19,7 +19,9 @@ from . import build as _build
 _LIB = None
 
 DDT_OK, DDT_ERR_INVALID_ARG, DDT_ERR_UNSUPPORTED, DDT_ERR_CUDA, DDT_ERR_INPUT = range(5)
-REQ_OK, REQ_BAD_PARENT, REQ_BAD_INDEX, REQ_WALK_LIMIT, REQ_BAD_PREFIX, REQ_BAD_LENGTH = range(6)
+REQ_OK, REQ_BAD_PARENT, REQ_BAD_INDEX, REQ_WALK_LIMIT, REQ_BAD_PREFIX, REQ_BAD_LENGTH, \
+    REQ_BAD_LP = range(7)
+FAULT_WAIT_TIMEOUT = 1
 DDT_F32, DDT_BF16 = 0, 1
 NUM_HEADS, D_LATENT, D_ROPE, MAX_Q_LEN = 64, 512, 64, 128
 
@@ -27,6 +29,7 @@ EXPORTED_SYMBOLS = (
     "ddt_tree_build", "ddt_build_mask", "ddt_verify_attn", "ddt_verify_attn_workspace_size",
     "ddt_verify_attn_num_splits", "ddt_tree_accept", "ddt_kv_compact", "ddt_accept_compact",
     "ddt_kv_write_block", "ddt_decode_step", "ddt_verify_attn_split_tail",
+    "ddt_selftest_bounded_wait",
     "ddt_verify_attn_split_tail_workspace_size",
     "ddt_status_str",
     "ddt_fault_flags", "ddt_version",
@@ -107,6 +110,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ddt_kv_write_block.restype = i32
     lib.ddt_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), V]
     lib.ddt_decode_step.restype = i32
+    lib.ddt_selftest_bounded_wait.argtypes = [ctypes.c_uint32, V, V]
+    lib.ddt_selftest_bounded_wait.restype = i32
     lib.ddt_status_str.argtypes = [i32]
     lib.ddt_status_str.restype = ctypes.c_char_p
     lib.ddt_fault_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -388,6 +393,14 @@ def decode_step_args(state: dict, step: dict, bufs: dict, softmax_scale: float,
 def decode_step(args: DecodeArgs, stream=None) -> None:
     """Launch one chained decode step (see decode_step_args)."""
     _check(load().ddt_decode_step(ctypes.byref(args), _stream(stream)), "ddt_decode_step")
+
+
+def selftest_bounded_wait(timeout_us: int = 2000, stream=None) -> torch.Tensor:
+    """Make one bounded wait give up (see ddt.h); returns the device flag it sets."""
+    gave_up = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    _check(load().ddt_selftest_bounded_wait(int(timeout_us), _ptr(gave_up), _stream(stream)),
+           "ddt_selftest_bounded_wait")
+    return gave_up
 
 
 def fault_flags(reset: bool = True) -> int:
