@@ -102,6 +102,9 @@ constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
 constexpr int kPBufBytes = kTK * 128;              // 64 rows x kTK keys bf16
 constexpr int kPBufs = DDT_VERIFY_P_BUFS;
 static_assert(kPBufs >= 1 && kPBufs <= 3, "one to three P buffers");
+// The epilogue stages half of a CTA's bf16 output (64 rows x 256 columns) in the P
+// buffers and stores it with TMA.
+static_assert(kPBufs * kPBufBytes >= 64 * 256 * 2, "P buffers hold half an output tile");
 constexpr int kVBlocks = kTK / 32;                 // 32-key V blocks per tile
 constexpr int kOffQ = 0;
 constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
@@ -238,7 +241,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_qrope,
                        const __grid_constant__ CUtensorMap tm_ckv_k,
                        const __grid_constant__ CUtensorMap tm_ckv_v,
-                       const __grid_constant__ CUtensorMap tm_krope, const VerifyParams p) {
+                       const __grid_constant__ CUtensorMap tm_krope,
+                       const __grid_constant__ CUtensorMap tm_out, const VerifyParams p) {
   using namespace va;
   const uint32_t rank = cluster_ctarank();
   const int cluster = static_cast<int>(blockIdx.x >> 1);
@@ -681,9 +685,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       const bool empty_row = !(l_row > 0.f);
       const float inv = empty_row ? 0.f : 1.f / l_row;
       const float lse_nat = empty_row ? -INFINITY : (m_use + __log2f(l_row)) * kLn2;
-      if (node_valid) {
-        const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
-        const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+      // bf16 output goes out through shared memory and TMA stores, so the
+      // tensor-memory reads (and the next item's first P V) need not wait for
+      // the global writes; fp32 outputs and split partials use plain stores.
+      const bool tma_out = node_valid && !p.write_partials && !p.out_f32;
+      if (tma_out) {
+        const int row0 = (b * Q + node) * 64;
+        uint8_t* stage = base + kOffP;
+        const uint32_t stage_addr = base_addr + kOffP;
 #pragma unroll 1
         for (int nh = 0; nh < 2; ++nh) {
 #pragma unroll 1
@@ -691,46 +700,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
             uint32_t o[32];
             tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
             tmem_wait_ld();
-            const int col = 256 * nh + 128 * hf + 32 * q;
-            if (p.write_partials) {
-              float4* dst = reinterpret_cast<float4*>(
-                  p.part_o + (static_cast<int64_t>(split + p.split_base) * rows_total + row) * 512 +
-                  col);
+            // columns 256 nh + 128 hf + 32 q ..: 64-column chunk 2 hf + q / 2 of this
+            // half, 16-byte units 4 (q & 1) .. + 3, 128-byte swizzle by row
+            uint8_t* rowp = stage + (2 * hf + (q >> 1)) * kStageBytes + m * 128;
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                     __uint_as_float(o[4 * v + 2]) * inv,
-                                     __uint_as_float(o[4 * v + 3]) * inv);
-            } else if (p.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                     __uint_as_float(o[4 * v + 2]) * inv,
-                                     __uint_as_float(o[4 * v + 3]) * inv);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * 512 + col);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(
-                    pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
-                    pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+            for (int v = 0; v < 4; ++v) {
+              const uint4 val = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * v]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+              *reinterpret_cast<uint4*>(rowp + (((4 * (q & 1) + v) ^ (m & 7)) << 4)) = val;
             }
           }
+          if (nh == 1) tc_fence_before_sync();  // every read of O is done
+          fence_proxy_async_smem();
+          named_barrier_sync(2, kSoftmaxThreads);
+          // O has been read: the next item's first P V may overwrite it.
+          if (nh == 1 && t == 0) mbar_arrive_cluster(o_free_leader);
+          if (t == 0) {
+            for (int c = 0; c < 4; ++c)
+              tma_store_3d(&tm_out, stage_addr + c * kStageBytes, 256 * nh + 64 * c, row0, 0);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging buffer may be written again
+          }
+          named_barrier_sync(2, kSoftmaxThreads);
         }
-        if (hf == 0) {
-          if (p.write_partials)
-            p.part_lse[static_cast<int64_t>(split + p.split_base) * rows_total + row] = lse_nat;
-          else if (p.lse) p.lse[row] = lse_nat;
+        if (hf == 0 && p.lse) p.lse[static_cast<int64_t>(row0) + m] = lse_nat;
+      } else {
+        if (node_valid) {
+          const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
+          const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+#pragma unroll 1
+          for (int nh = 0; nh < 2; ++nh) {
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
+              tmem_wait_ld();
+              const int col = 256 * nh + 128 * hf + 32 * q;
+              float4* dst =
+                  p.write_partials
+                      ? reinterpret_cast<float4*>(
+                            p.part_o +
+                            (static_cast<int64_t>(split + p.split_base) * rows_total + row) * 512 +
+                            col)
+                      : reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                     __uint_as_float(o[4 * v + 2]) * inv,
+                                     __uint_as_float(o[4 * v + 3]) * inv);
+            }
+          }
+          if (hf == 0) {
+            if (p.write_partials)
+              p.part_lse[static_cast<int64_t>(split + p.split_base) * rows_total + row] = lse_nat;
+            else if (p.lse) p.lse[row] = lse_nat;
+          }
         }
+        // O has been read: the next item's first P V may overwrite it.
+        tc_fence_before_sync();
+        named_barrier_sync(2, kSoftmaxThreads);
+        if (t == 0) mbar_arrive_cluster(o_free_leader);
       }
-      // O has been read: the next item's first P V may overwrite it.
-      tc_fence_before_sync();
-      named_barrier_sync(2, kSoftmaxThreads);
-      if (t == 0) mbar_arrive_cluster(o_free_leader);
     }
+    if (t == 0) bulk_wait_group0();  // this CTA's output stores have completed
   }
 
   // All MMAs of the pair are complete here (the softmax warps waited for the
@@ -855,7 +890,7 @@ namespace {
 ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int write_partials,
                        int split_base, float* part_o, float* part_lse, cudaStream_t stream) {
   using namespace va;
-  CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope;
+  CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out;
   const uint64_t rows_q = static_cast<uint64_t>(a.q_len) * 64;
   const uint64_t B = static_cast<uint64_t>(a.B);
   const uint64_t cap = static_cast<uint64_t>(a.capacity);
@@ -864,6 +899,12 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
             make_map(&m_ckv_k, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, kKH) &&
             make_map(&m_ckv_v, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 32) &&
             make_map(&m_krope, a.k_rope, 64, cap, B, a.kr_row_stride * 2, a.kr_batch_stride * 2, kKH);
+  // bf16 output rows [B * q_len * 64, 512], stored in 64 x 64 boxes by the epilogue
+  const uint64_t out_rows = static_cast<uint64_t>(a.B) * a.q_len * 64;
+  if (!write_partials && a.out_dtype == DDT_BF16)
+    ok = ok && make_map(&m_out, a.out, 512, out_rows, 1, 512 * 2, out_rows * 512 * 2, 64);
+  else
+    m_out = m_qlat;  // not read
   if (!ok) return DDT_ERR_INVALID_ARG;
   if (ensure_smem_limit(reinterpret_cast<const void*>(verify_attn_kernel), kSmemBytes, 1) !=
       cudaSuccess)
@@ -892,7 +933,7 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
   const int64_t slots = device_sm_count() / 2 > 0 ? device_sm_count() / 2 : 1;
   const int64_t grid = 2 * (items < slots ? items : slots);
   verify_attn_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
-      m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, p);
+      m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out, p);
   return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
