@@ -133,12 +133,17 @@ def _compare(chain, ref, c_ref, k_ref, P_ref, root_ref):
     assert np.array_equal(s["root_token"].cpu().numpy(), root_ref)
 
 
-@pytest.mark.parametrize("B,Q,D,K,n", [(4, 17, 15, 4, 3), (2, 33, 15, 8, 4)])
-def test_decode_chain_eager_and_graph(B, Q, D, K, n):
+@pytest.mark.parametrize("B,Q,D,K,n,P0", [(4, 17, 15, 4, 3, [100, 257, 600, 31]),
+                                           (2, 33, 15, 8, 4, [100, 257]),
+                                           (1, 17, 15, 8, 2, [2000])])
+def test_decode_chain_eager_and_graph(B, Q, D, K, n, P0):
+    """Few work items for 148 SMs, so every case's verify runs split-KV with the
+    caller's workspace, inside the chain and inside the graph; the last case (one
+    request, a 2000-row prefix) splits its keys six ways."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     steps = _steps(7 + Q, B, Q, D, K, n)
-    P0 = np.array([100, 257, 600, 31][:B], dtype=np.int32)
+    P0 = np.array(P0, dtype=np.int32)
     cap = int(P0.max()) + (n + 1) * Q
     g = inputs.normal(inputs.stream_base(3, 96, 0), B * cap * (DL + DR))
     bits = inputs.to_bf16_bits(g).reshape(B, cap, DL + DR)
@@ -149,6 +154,7 @@ def test_decode_chain_eager_and_graph(B, Q, D, K, n):
     assert any((r["alen"] > 1).any() for r in ref)
 
     chain = Chain(steps, c_kv, k_rope, P0, root, Q, scale, max_prefix=cap - Q)
+    assert all("workspace" in b for b in chain.bufs)
     ddt.fault_flags(reset=True)
     chain.run()
     _compare(chain, ref, c_ref, k_ref, P_ref, root_ref)

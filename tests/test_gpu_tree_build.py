@@ -121,3 +121,14 @@ def test_tree_build_feeds_tree_accept():
     assert np.array_equal(path.cpu().numpy(), want[0])
     assert np.array_equal(alen.cpu().numpy(), want[1])
     assert (alen.cpu().numpy() > 1).any()
+
+
+def test_tree_build_weights_that_overflow():
+    """Finite log-probs whose sums overflow to -inf: the weights of whole subtrees
+    become -inf and tie; both sides order them by insertion all the same."""
+    lp, tok, root = _draft(84, 4, 12, 4)
+    lp[:, 1:3, :] = np.float32(-3.0e38)  # depth-3 weights: -6e38 rounds to -inf
+    lp[1, 0, 1:] = np.float32(-3.0e38)
+    g = _check(lp, tok, root, 65)
+    assert (g["status"] == 0).all() and (g["n_nodes"] == 65).all()
+    assert (np.isinf(g["logw"]).sum(axis=1) >= 44).all()
