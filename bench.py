@@ -609,6 +609,58 @@ def accept_sweep() -> int:
     return 0
 
 
+def compact_scale() -> int:
+    """kv_compact on batches large enough to be bound by HBM rather than by launch
+    latency: 1024 requests, q_len 128, 256-row prefixes, separate contiguous caches
+    (453 MB), with accepted paths that move most rows: the reversed block (alen 128,
+    keep[i] = 127 - i: every row moves) and every second node (alen 64, keep[i] = 2 i:
+    63 rows move).  Bytes per call = every moved row read once and written once
+    (1152 B each).  20 calls per CUDA graph, L2 flushed before each (flush time
+    subtracted), median of 5.  One JSON line."""
+    import torch
+
+    from tree_speculative_decoding_05_b200 import ddt
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = measured_peaks()
+    B, Q, P = 1024, 128, 256
+    cap = P + Q
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(12)
+    bits = lambda d: torch.randint(-32768, 32768, (B, cap, d), dtype=torch.int32, device=dev,
+                                   generator=gen).to(torch.int16).view(torch.bfloat16)
+    c_kv, k_rope = bits(DL), bits(DR)
+    prefix = torch.full((B,), P, dtype=torch.int32, device=dev)
+    newp = torch.empty_like(prefix)
+    status = torch.empty_like(prefix)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, alen_v, keep in (("reversed block", Q, [Q - 1 - i for i in range(Q)]),
+                               ("every second node", Q // 2, [2 * i for i in range(Q // 2)])):
+        row = np.zeros(Q, dtype=np.int32)
+        row[:alen_v] = keep
+        path = torch.from_numpy(np.tile(row, (B, 1))).to(dev)
+        alen = torch.full((B,), alen_v, dtype=torch.int32, device=dev)
+        moved = sum(1 for i, k in enumerate(keep) if k != i)
+        fn = lambda: ddt.kv_compact(c_kv, k_rope, prefix, path, alen, new_prefix_lens=newp,
+                                    status=status)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        assert bool((status == 0).all()), "kv_compact status"
+        us = graph_time_us(fn, 20, flush=flush)
+        nbytes = 2.0 * B * moved * (DL + DR) * 2
+        gbs = nbytes / (us * 1e-6) / 1e9
+        res[name] = {"alen": alen_v, "rows_moved_per_request": moved, "bytes_per_call": nbytes,
+                     "us_per_call": us, "gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
+    print(json.dumps({"kv_compact_at_scale": res, "requests": B, "q_len": Q, "prefix": P,
+                      "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
+                      "timing": "20 calls per CUDA graph, L2 flushed before each call "
+                                "(flush subtracted), median of 5"}), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -628,6 +680,9 @@ def main(argv=None) -> int:
     ap.add_argument("--accept-sweep", action="store_true",
                     help="tree_accept alone over streams {1, 8, 64} x budget {8, 32} (the grid "
                          "the pages report), graph-timed; one JSON line")
+    ap.add_argument("--compact-scale", action="store_true",
+                    help="kv_compact alone on 1024 requests x q_len 128 with paths that move "
+                         "most rows (HBM-bound, not latency-bound); one JSON line")
     ap.add_argument("--shard", choices=["replicas", "lpt"], default="replicas",
                     help="with several GPUs: every rank runs its own batch of the workload "
                          "(replicas, weak scaling) or the ranks split one batch by request "
@@ -645,6 +700,8 @@ def main(argv=None) -> int:
         return per_call_report(args)
     if args.accept_sweep:
         return accept_sweep()
+    if args.compact_scale:
+        return compact_scale()
     if args.impl == "reference":
         if rank != 0:
             return 0

@@ -131,6 +131,24 @@ def test_kv_compact_bit_exact(kind, Q):
         assert np.array_equal(g, r), name
 
 
+def test_kv_compact_at_scale():
+    """The benchmark's at-scale patterns on 512 requests x q_len 128: the reversed
+    block (every row moves, each one onto a row another request row reads) and every
+    second node, mixed with identity rows, bit for bit against the oracle."""
+    B, Q = 512, 128
+    c_kv, k_rope, Pv, path, alen, cap = _compact_case(B, Q, [256] * B, 91, "identity")
+    for b in range(B):
+        if b % 3 == 0:
+            path[b, :] = np.arange(Q - 1, -1, -1); alen[b] = Q
+        elif b % 3 == 1:
+            path[b, :64] = 2 * np.arange(64); alen[b] = 64
+    ref = oracle.kv_compact(c_kv, k_rope, Pv, path, alen, capacity=cap)
+    got = _run_compact(c_kv, k_rope, Pv, path, alen, cap)
+    for g, r, name in zip(got, ref, ("c_kv", "k_rope", "new_prefix", "status")):
+        assert np.array_equal(g, r), name
+    assert (ref[3] == 0).all()
+
+
 def test_kv_compact_race_pattern_and_errors():
     """keep = [0, 2, 3] (the racing pattern) plus malformed requests."""
     B, Q = 4, 8

@@ -157,6 +157,17 @@ constexpr int kLatVec = DDT_D_LATENT * 2 / 16;  // 16-byte vectors per latent ro
 constexpr int kRopeVec = DDT_D_ROPE * 2 / 16;   // per rope row (8)
 constexpr int kRowVec = kLatVec + kRopeVec;
 
+// Asynchronous 16-byte copy global -> shared (cp.async, L2 only): a thread can have
+// all of its copies in flight at once instead of one load per loop iteration.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Moves rows P+keep[i] -> P+i (i < alen) of request b, both caches, through
 // shared memory: every moving row is read before any is written.  Called by all
 // kCompactThreads threads of the CTA; s_rows holds alen * kRowVec vectors.
@@ -167,13 +178,15 @@ __device__ void compact_rows(uint16_t* __restrict__ c_kv, uint16_t* __restrict__
   const uint4* kr_b = reinterpret_cast<const uint4*>(k_rope + b * kr_bs);
   const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;  // row strides in 16-byte vectors
   const int total = alen * kRowVec;
-  // Phase 1: every moving row into shared memory.
+  // Phase 1: every moving row into shared memory, all copies in flight together.
   for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
     const int i = idx / kRowVec, v = idx - i * kRowVec;
     if (s_keep[i] == i) continue;
     const int64_t src_row = P + s_keep[i];
-    s_rows[idx] = (v < kLatVec) ? ckv_b[src_row * ckv_rv + v] : kr_b[src_row * kr_rv + (v - kLatVec)];
+    cp_async16(&s_rows[idx], (v < kLatVec) ? ckv_b + (src_row * ckv_rv + v)
+                                           : kr_b + (src_row * kr_rv + (v - kLatVec)));
   }
+  cp_async_wait_all();
   __syncthreads();
   // Phase 2: write rows P .. P+alen-1 (only those that move).
   uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
