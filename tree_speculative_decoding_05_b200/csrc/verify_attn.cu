@@ -19,11 +19,12 @@
 //     lanes: lanes 0-63 hold columns [0, N/2) and lanes 64-127 columns [N/2, N).
 //   * S = Q K^T per 128-key tile: 36 MMAs of N = 128, K = 16 (576 = 9 chunks of
 //     64).  Q (64 rows x 576, 72 KB per CTA) stays in shared memory; each CTA
-//     stages its half of the keys (64 keys x 64 dims = 8 KB per stage).
+//     stages its half of the keys, two 64-dim chunks per ring stage (64 keys x
+//     128 dims = 16 KB, one commit per 8 MMAs).
 //   * O += P V per tile: 16 MMAs of N = 256, K = 16 into two fp32 accumulators
 //     covering the 512 latent columns (128 TMEM columns each per CTA).  V is the
 //     same c_kv rows read as an MN-major operand (each CTA stages 128 latent
-//     columns x 32 keys = 8 KB per stage).
+//     columns x 64 keys = 16 KB per stage, one commit per 4 MMAs).
 //   * TMEM per CTA: four S buffers (4 x 64 cols) + O (256 cols) = all 512
 //     columns; four S buffers let S = Q K^T run up to three tiles ahead of the
 //     softmax.
@@ -83,12 +84,28 @@ constexpr int kStageBytes = 8192;                  // Q chunk, V stage, P chunk:
 constexpr int kTK = DDT_VERIFY_TILE_KEYS;
 static_assert(kTK == 128 || kTK == 256, "KV tiles of 128 or 256 rows");
 constexpr int kKH = kTK / 2;
-constexpr int kKStageBytes = kKH * 128;            // K stage: kKH keys x 64 dims
+// K stage: kKStageChunks 64-dim chunks of kKH keys, committed as one unit after
+// their 4 * kKStageChunks MMAs; a tile's 9 chunks (8 latent + 1 rope) fill
+// kKStagesPerTile stages, the last one partly when the stages hold two chunks.
+// Fewer, larger stages mean fewer commits and barrier round trips per tile: with
+// 128-key tiles, two-chunk K stages and 64-key V stages (the defaults) run the
+// 64 x 33 x 4096 workload 6 % faster than one-chunk K and 32-key V stages over
+// the same ring bytes.
+#ifndef DDT_VERIFY_K_STAGE_CHUNKS
+#define DDT_VERIFY_K_STAGE_CHUNKS (DDT_VERIFY_TILE_KEYS == 128 ? 2 : 1)
+#endif
+constexpr int kKStageChunks = DDT_VERIFY_K_STAGE_CHUNKS;
+static_assert(kKStageChunks == 1 || kKStageChunks == 2, "K stages of one or two chunks");
+constexpr int kKChunkBytes = kKH * 128;            // kKH keys x 64 dims
+constexpr int kKStageBytes = kKChunkBytes * kKStageChunks;
 #ifndef DDT_VERIFY_K_STAGES
-#define DDT_VERIFY_K_STAGES (DDT_VERIFY_TILE_KEYS == 128 ? 4 : 2)
+#define DDT_VERIFY_K_STAGES (DDT_VERIFY_TILE_KEYS == 128 && DDT_VERIFY_K_STAGE_CHUNKS == 1 ? 4 : 2)
+#endif
+#ifndef DDT_VERIFY_V_KEYS
+#define DDT_VERIFY_V_KEYS 64
 #endif
 #ifndef DDT_VERIFY_V_STAGES
-#define DDT_VERIFY_V_STAGES 6
+#define DDT_VERIFY_V_STAGES (DDT_VERIFY_V_KEYS == 32 ? 6 : 3)
 #endif
 // P buffers in shared memory: the softmax of tile G writes P into buffer
 // G % kPBufs once the P V of tile G - kPBufs has read it.
@@ -97,19 +114,25 @@ constexpr int kKStageBytes = kKH * 128;            // K stage: kKH keys x 64 dim
 #endif
 constexpr int kKStages = DDT_VERIFY_K_STAGES;      // each of the two K rings (even / odd tiles)
 constexpr int kVStages = DDT_VERIFY_V_STAGES;      // V ring (feeds O += P V)
+// V stage: kVKeys cache rows x 128 latent columns (this CTA's half of one N = 256
+// accumulator), committed as one unit after its kVKeys / 16 MMAs.
+constexpr int kVKeys = DDT_VERIFY_V_KEYS;
+static_assert(kVKeys == 32 || kVKeys == 64, "V stages of 32 or 64 keys");
+constexpr int kVStageBytes = kVKeys * 256;
 constexpr int kQChunks = 9;                        // 8 latent chunks + 1 rope chunk
 constexpr int kQBytes = kQChunks * kStageBytes;    // 64 rows x 576 bf16
+constexpr int kKStagesPerTile = (kQChunks + kKStageChunks - 1) / kKStageChunks;
 constexpr int kPBufBytes = kTK * 128;              // 64 rows x kTK keys bf16
 constexpr int kPBufs = DDT_VERIFY_P_BUFS;
 static_assert(kPBufs >= 1 && kPBufs <= 3, "one to three P buffers");
 // The epilogue stages half of a CTA's bf16 output (64 rows x 256 columns) in the P
 // buffers and stores it with TMA.
 static_assert(kPBufs * kPBufBytes >= 64 * 256 * 2, "P buffers hold half an output tile");
-constexpr int kVBlocks = kTK / 32;                 // 32-key V blocks per tile
+constexpr int kVBlocks = kTK / kVKeys;             // V blocks per tile
 constexpr int kOffQ = 0;
 constexpr int kOffKRing = kOffQ + kQBytes;           // two rings of kKStages
 constexpr int kOffVRing = kOffKRing + kQKIss * kKStages * kKStageBytes;
-constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
+constexpr int kOffP = kOffVRing + kVStages * kVStageBytes;
 constexpr int kOffRedMax = kOffP + kPBufs * kPBufBytes;  // float[2][128]
 constexpr int kOffRedL = kOffRedMax + 2 * 128 * 4;     // float[128]
 constexpr int kMaxSortedB = 512;  // requests ordered by length (larger B: natural order)
@@ -377,13 +400,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         for (int jj = 0; jj < it.ntile; ++jj, ++G) {
           if (static_cast<int>(G % kQKIss) != g) continue;
           const int key0 = tile_start(it, it.t0 + jj) + key_half;
-          for (int c = 0; c < kQChunks; ++c) {
+          for (int sc = 0; sc < kKStagesPerTile; ++sc) {
+            const int c0 = sc * kKStageChunks;
+            const int nch = kQChunks - c0 < kKStageChunks ? kQChunks - c0 : kKStageChunks;
             mbar_wait(bar(empty0 + r.stage), r.phase ^ 1u, abort_flag);
-            if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * kKStageBytes);
+            if (leader) mbar_arrive_expect_tx_local(bar(full0 + r.stage), 2 * nch * kKChunkBytes);
             const uint32_t fb = map_to_rank(bar(full0 + r.stage), 0);
-            const uint32_t dst = ring + r.stage * kKStageBytes;
-            if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, it.b);
-            else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, it.b);
+            for (int u = 0; u < nch; ++u) {
+              const int c = c0 + u;
+              const uint32_t dst = ring + r.stage * kKStageBytes + u * kKChunkBytes;
+              if (c < 8) tma_load_3d_pair(dst, &tm_ckv_k, fb, 64 * c, key0, it.b);
+              else tma_load_3d_pair(dst, &tm_krope, fb, 0, key0, it.b);
+            }
             r.advance(kKStages);
           }
         }
@@ -402,15 +430,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         if (!it.valid) continue;
         for (int jj = 0; jj < it.ntile; ++jj) {
           for (int kb = 0; kb < kVBlocks; ++kb) {
-            const int key0 = tile_start(it, it.t0 + jj) + 32 * kb;
+            const int key0 = tile_start(it, it.t0 + jj) + kVKeys * kb;
             for (int nh = 0; nh < 2; ++nh) {
               mbar_wait(bar(kBarVEmpty + r.stage), r.phase ^ 1u, abort_flag);
-              if (leader) mbar_arrive_expect_tx_local(bar(kBarVFull + r.stage), 2 * kStageBytes);
+              if (leader) mbar_arrive_expect_tx_local(bar(kBarVFull + r.stage), 2 * kVStageBytes);
               const uint32_t fb = map_to_rank(bar(kBarVFull + r.stage), 0);
               const int x0 = 256 * nh + 128 * static_cast<int>(rank);
-              const uint32_t dst = sVRing + r.stage * kStageBytes;
+              const uint32_t dst = sVRing + r.stage * kVStageBytes;
               tma_load_3d_pair(dst, &tm_ckv_v, fb, x0, key0, it.b);
-              tma_load_3d_pair(dst + 4096, &tm_ckv_v, fb, x0 + 64, key0, it.b);
+              tma_load_3d_pair(dst + kVStageBytes / 2, &tm_ckv_v, fb, x0 + 64, key0, it.b);
               r.advance(kVStages);
             }
           }
@@ -445,14 +473,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
             tc_fence_after_sync();
           }
           const uint32_t d = tmem + kTmemS + static_cast<uint32_t>(kSCols * sbuf);
-          for (int c = 0; c < kQChunks; ++c) {
+          for (int sc = 0; sc < kKStagesPerTile; ++sc) {
+            const int c0 = sc * kKStageChunks;
+            const int nch = kQChunks - c0 < kKStageChunks ? kQChunks - c0 : kKStageChunks;
             mbar_wait(bar(full0 + r.stage), r.phase, abort_flag);
-            const uint32_t a0 = sQ + c * kStageBytes;
-            const uint32_t b0 = ring + r.stage * kKStageBytes;
+            for (int u = 0; u < nch; ++u) {
+              const int c = c0 + u;
+              const uint32_t a0 = sQ + c * kStageBytes;
+              const uint32_t b0 = ring + r.stage * kKStageBytes + u * kKChunkBytes;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
-                             smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
+              for (int ks = 0; ks < 4; ++ks)
+                mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
+                               smem_desc_sw128(b0 + 32 * ks, 16, 1024), kIdescQK, (c | ks) != 0);
+            }
             mma_commit<2>(bar(empty0 + r.stage), 0x3);
             r.advance(kKStages);
           }
@@ -490,12 +523,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
             for (int nh = 0; nh < 2; ++nh) {
               mbar_wait(bar(kBarVFull + r.stage), r.phase, abort_flag);
               const uint32_t d = tmem + kTmemO + 128u * static_cast<uint32_t>(nh);
-              const uint32_t a0 = sP + pb * kPBufBytes + (kb >> 1) * kStageBytes + (kb & 1) * 64;
-              const uint32_t b0 = sVRing + r.stage * kStageBytes;
+              // P keys [kVKeys kb, + kVKeys): 64-key chunk, then 2 bytes per key in its row
+              const int pk0 = kVKeys * kb;
+              const uint32_t a0 = sP + pb * kPBufBytes + (pk0 >> 6) * kStageBytes + (pk0 & 63) * 2;
+              const uint32_t b0 = sVRing + r.stage * kVStageBytes;
 #pragma unroll
-              for (int ks = 0; ks < 2; ++ks)
+              for (int ks = 0; ks < kVKeys / 16; ++ks)
                 mma_bf16_ss<2>(d, smem_desc_sw128(a0 + 32 * ks, 16, 1024),
-                               smem_desc_sw128(b0 + 2048 * ks, 4096, 1024), kIdescPV,
+                               smem_desc_sw128(b0 + 2048 * ks, kVStageBytes / 2, 1024), kIdescPV,
                                !(jj == 0 && kb == 0 && ks == 0));
               mma_commit<2>(bar(kBarVEmpty + r.stage), 0x3);
               r.advance(kVStages);
@@ -897,7 +932,7 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
   bool ok = make_map(&m_qlat, a.q_lat, 512, rows_q, B, 512 * 2, rows_q * 512 * 2, 64) &&
             make_map(&m_qrope, a.q_rope, 64, rows_q, B, 64 * 2, rows_q * 64 * 2, 64) &&
             make_map(&m_ckv_k, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, kKH) &&
-            make_map(&m_ckv_v, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, 32) &&
+            make_map(&m_ckv_v, a.c_kv, 512, cap, B, a.ckv_row_stride * 2, a.ckv_batch_stride * 2, kVKeys) &&
             make_map(&m_krope, a.k_rope, 64, cap, B, a.kr_row_stride * 2, a.kr_batch_stride * 2, kKH);
   // bf16 output rows [B * q_len * 64, 512], stored in 64 x 64 boxes by the epilogue
   const uint64_t out_rows = static_cast<uint64_t>(a.B) * a.q_len * 64;
