@@ -28,15 +28,20 @@
 // key.  A register holds an order-preserving 32-bit key of the weight (larger
 // weight, larger key; equal weights, equal keys; 0 = empty slot); the exact
 // weight and the (depth, rank, parent) of each slot sit in shared memory.  A
-// pick is two warp-wide hardware reductions: the maximum key, then the
-// smallest slot holding it — no heap and no shuffle tree.  The log-probs and tokens a
+// pick is a lane-local maximum over the lane's key registers (fully unrolled,
+// so the keys never leave registers) and two warp-wide hardware reductions:
+// the maximum key, then the smallest slot holding it — no heap, no shuffle tree
+// and no memory access before the winner is known.  The log-probs and tokens a
 // build can touch (depth rows < min(D, q_len-1), ranks < min(K, q_len)) are
-// staged in shared memory first, so no pick waits on global memory.  The
-// weights use explicitly rounded float32 adds and subtracts (__fadd_rn /
-// __fsub_rn), which the compiler may neither contract nor reorder, so the
-// result is bit-identical to any float32 evaluation of the same expressions.
-// After the expansion the lanes build, one node each, the visibility words,
-// the retrieve pointers and the padding, and write everything coalesced.
+// staged in shared memory first, in the same pass that checks every log-prob
+// for finiteness, so no pick waits on global memory.  The weights use
+// explicitly rounded float32 adds and subtracts (__fadd_rn / __fsub_rn), which
+// the compiler may neither contract nor reorder, so the result is bit-identical
+// to any float32 evaluation of the same expressions.  Each new node is linked
+// as the newest child of its parent as it is created, which gives the retrieve
+// pointers (first child, next sibling) without a search.  After the expansion
+// the lanes build, one node each, the visibility words and the padding, and
+// write everything coalesced.
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -50,6 +55,10 @@ namespace ddt {
 namespace tb {
 // Dynamic shared memory bound: rows < q_len-1, ranks < q_len, float + int each.
 constexpr int kMaxStageBytes = (DDT_MAX_Q_LEN - 1) * DDT_MAX_Q_LEN * 8;
+// Candidate slots: at most 1 + 2 (q_len - 1) insertions; key registers per lane.
+constexpr int kMaxSlots = 2 * DDT_MAX_Q_LEN;
+constexpr int kKeyRegs = kMaxSlots / 32;
+static_assert(kMaxSlots % 32 == 0, "whole key registers");
 }  // namespace tb
 
 // Order-preserving key of a weight: larger weight, larger key; -0 and +0 map to
@@ -58,6 +67,14 @@ __device__ __forceinline__ uint32_t weight_key(float w) {
   uint32_t u = __float_as_uint(w);
   if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Sets key register `reg` of a lane's candidate keys (reg is warp-uniform; the
+// unrolled compare keeps every index a constant, so the array stays in registers).
+__device__ __forceinline__ void set_key(uint32_t (&ck)[tb::kKeyRegs], int reg, uint32_t key) {
+#pragma unroll
+  for (int j = 0; j < tb::kKeyRegs; ++j)
+    if (j == reg) ck[j] = key;
 }
 
 __global__ void __launch_bounds__(32) tree_build_kernel(
@@ -74,9 +91,11 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   __shared__ int32_t s_ntok[DDT_MAX_Q_LEN];
   __shared__ int32_t s_dep[DDT_MAX_Q_LEN];
   __shared__ float s_lw[DDT_MAX_Q_LEN];
-  __shared__ uint32_t s_ck[2 * DDT_MAX_Q_LEN];  // candidate order key per slot, 0 = empty
-  __shared__ float s_cw[2 * DDT_MAX_Q_LEN];     // candidate weight per slot
-  __shared__ int32_t s_cm[2 * DDT_MAX_Q_LEN];   // candidate depth | rank << 8 | parent << 16
+  __shared__ int32_t s_first[DDT_MAX_Q_LEN];  // first child (-1: none)
+  __shared__ int32_t s_next[DDT_MAX_Q_LEN];   // next sibling (-1: none)
+  __shared__ int32_t s_last[DDT_MAX_Q_LEN];   // newest child so far (-1: none)
+  __shared__ float s_cw[tb::kMaxSlots];       // candidate weight per slot
+  __shared__ int32_t s_cm[tb::kMaxSlots];     // candidate depth | rank << 8 | parent << 16
 
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
@@ -84,15 +103,25 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   const float* L = lp + b * DK;
   const int32_t* T = tok + b * DK;
 
-  // Every log-prob must be finite (a NaN would make the arg-max order-dependent).
+  // One pass over the drafts: every log-prob must be finite (a NaN would make
+  // the arg-max order-dependent), and the entries a build can read are staged.
   bool bad = false;
-  for (int64_t e = lane; e < DK; e += 32) bad |= !isfinite(L[e]);
+#pragma unroll 4
+  for (int64_t e = lane; e < DK; e += 32) {
+    const float v = L[e];
+    bad |= !isfinite(v);
+    const int64_t d = e / K;
+    const int64_t r = e - d * K;
+    if (d < Dp && r < Kp) {
+      s_lp[d * Kp + r] = v;
+      s_tok[d * Kp + r] = T[e];
+    }
+  }
   bad = __any_sync(0xffffffffu, bad);
-
-  for (int e = lane; e < Dp * Kp; e += 32) {
-    const int d = e / Kp, r = e - d * Kp;
-    s_lp[e] = L[static_cast<int64_t>(d) * K + r];
-    s_tok[e] = T[static_cast<int64_t>(d) * K + r];
+  for (int i = lane; i < q_len; i += 32) {
+    s_first[i] = -1;
+    s_next[i] = -1;
+    s_last[i] = -1;
   }
   if (lane == 0) {
     s_par[0] = -1;
@@ -102,36 +131,43 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   }
   __syncwarp();
 
-  // Candidate slots in insertion order; lane l scans slots l, l + 32, ...
+  // Candidate keys: slot s in lane s % 32, register s / 32 (0 = empty).  Every
+  // register index below is a compile-time constant, so ck stays in registers.
+  uint32_t ck[tb::kKeyRegs];
+#pragma unroll
+  for (int j = 0; j < tb::kKeyRegs; ++j) ck[j] = 0u;
   int n_slots = 0;
-  auto insert = [&](float w, int meta) {  // one slot, written by lane 0
-    if (lane == 0) {
-      s_ck[n_slots] = weight_key(w);
-      s_cw[n_slots] = w;
-      s_cm[n_slots] = meta;
-    }
-    ++n_slots;
-  };
-  if (!bad && q_len > 1) insert(__fadd_rn(0.0f, s_lp[0]), 1 | (0 << 8) | (0 << 16));
+  // Inserts one candidate: its key in the slot's lane, weight and metadata by lane 0.
+#define DDT_TB_INSERT(w_, meta_)                                   \
+  do {                                                             \
+    const int sl_ = n_slots++;                                     \
+    const float wv_ = (w_);                                        \
+    if (lane == (sl_ & 31)) set_key(ck, sl_ >> 5, weight_key(wv_)); \
+    if (lane == 0) {                                               \
+      s_cw[sl_] = wv_;                                             \
+      s_cm[sl_] = (meta_);                                         \
+    }                                                              \
+  } while (0)
+  if (!bad && q_len > 1) DDT_TB_INSERT(__fadd_rn(0.0f, s_lp[0]), 1 | (0 << 8) | (0 << 16));
   __syncwarp();
 
   int n = 1;
   while (n < q_len) {
-    // Lane-local best: a lane's slots ascend, so a later equal key never wins.
+    // Lane-local best: a lane's slots ascend with the register index, so a later
+    // equal key never wins.
     uint32_t bk = 0u;
     uint32_t bs = 0xffffffffu;
-    for (int sl = lane; sl < n_slots; sl += 32) {
-      const uint32_t key = s_ck[sl];
-      if (key > bk) {
-        bk = key;
-        bs = static_cast<uint32_t>(sl);
+#pragma unroll
+    for (int j = 0; j < tb::kKeyRegs; ++j) {
+      if (ck[j] > bk) {
+        bk = ck[j];
+        bs = static_cast<uint32_t>(j * 32 + lane);
       }
     }
     const uint32_t kmax = __reduce_max_sync(0xffffffffu, bk);
     if (kmax == 0u) break;  // no candidate left
     const uint32_t win = __reduce_min_sync(0xffffffffu, bk == kmax ? bs : 0xffffffffu);
-    __syncwarp();  // every lane has read the keys before the winner's is cleared
-    if (lane == 0) s_ck[win] = 0u;
+    if (lane == static_cast<int>(win & 31u)) set_key(ck, static_cast<int>(win >> 5), 0u);
     const float bw = s_cw[win];
     const int meta = s_cm[win];
     const int d = meta & 0xff, r = (meta >> 8) & 0xff, par = meta >> 16;
@@ -141,15 +177,21 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
       s_ntok[node] = s_tok[(d - 1) * Kp + r];
       s_dep[node] = d;
       s_lw[node] = bw;
+      // node is the newest child of par: the first one, or the next sibling of the last
+      const int prev = s_last[par];
+      if (prev < 0) s_first[par] = node;
+      else s_next[prev] = node;
+      s_last[par] = node;
     }
     if (n == q_len) break;  // budget reached: nothing more will be picked
-    if (d < D) insert(__fadd_rn(bw, s_lp[d * Kp]), (d + 1) | (0 << 8) | (node << 16));
+    if (d < D) DDT_TB_INSERT(__fadd_rn(bw, s_lp[d * Kp]), (d + 1) | (0 << 8) | (node << 16));
     if (r + 1 < K) {
       const float w = __fadd_rn(__fsub_rn(bw, s_lp[(d - 1) * Kp + r]), s_lp[(d - 1) * Kp + r + 1]);
-      insert(w, d | ((r + 1) << 8) | (par << 16));
+      DDT_TB_INSERT(w, d | ((r + 1) << 8) | (par << 16));
     }
-    __syncwarp();  // the new slots are visible to every lane
+    __syncwarp();  // the new slots' weights and metadata are visible to every lane
   }
+#undef DDT_TB_INSERT
   __syncwarp();
 
   // Per node: padding, retrieve pointers, visibility words; coalesced writes.
@@ -164,17 +206,8 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
       t = s_ntok[i];
       dd = s_dep[i];
       w = s_lw[i];
-      for (int c = i + 1; c < n; ++c)
-        if (s_par[c] == i) {
-          first = c;
-          break;
-        }
-      if (i > 0)
-        for (int c = i + 1; c < n; ++c)
-          if (s_par[c] == p) {
-            sib = c;
-            break;
-          }
+      first = s_first[i];
+      sib = s_next[i];  // -1 for the root, which is no one's child
       for (int a = i, steps = 0; a >= 0 && steps <= i; a = s_par[a], ++steps) {
         if (a < 64) w0 |= 1ull << a;
         else w1 |= 1ull << (a - 64);
