@@ -78,7 +78,7 @@ static_assert(kQKIss == 2 || kQKIss == 3, "two or three S issuers");
 // issuer, 8 K producer 1, 9 S issuer 1, 10 K producer 2, 11 S issuer 2.
 constexpr int kThreads = 32 * (6 + 2 * kQKIss);
 constexpr int kSoftmaxThreads = 128;
-constexpr int kStageBytes = 8192;                  // Q chunk, V stage, P chunk: 64 x 128 B
+constexpr int kStageBytes = 8192;                  // Q chunk, P chunk, output box: 64 x 128 B
 // KV tile: kTK cache rows per tile; each CTA of the pair stages kKH of them for
 // S = Q K^T (the pair's MMA has N = kTK).
 constexpr int kTK = DDT_VERIFY_TILE_KEYS;
