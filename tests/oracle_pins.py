@@ -321,6 +321,31 @@ def pin_compact_golden(orc):
         assert np.array_equal(kr2[0], np.array(case["k_rope"], np.uint16)), case["name"]
 
 
+def pin_compact_closed_forms(orc):
+    """Whole-block keep lists whose result has a closed form: row P + i takes the old
+    row P + keep[i] for i < alen, every other row is unchanged ([Race Conditions] "The
+    Cache Compaction Problem": the gather reads old rows, so every read precedes every
+    write).  The reversed block makes every destination a source of another row; every
+    second node reads ahead of each write."""
+    Q, P, extra = 16, 5, 3
+    cap = P + Q + extra
+    rows = np.arange(cap, dtype=np.uint16)
+    c_kv = np.stack([rows * 7 + 1, rows * 7 + 2], axis=-1)[None].astype(np.uint16)
+    k_rope = (rows * 3 + 9)[None, :, None].astype(np.uint16)
+    for keep in (list(range(Q - 1, -1, -1)), [2 * i for i in range(Q // 2)], [0], list(range(Q))):
+        alen = len(keep)
+        path = np.full((1, Q), -1, np.int32)
+        path[0, :alen] = keep
+        ckv2, kr2, newp, status = orc.kv_compact(c_kv, k_rope, np.array([P], np.int32), path,
+                                                 np.array([alen], np.int32), capacity=cap)
+        want_c, want_r = c_kv.copy(), k_rope.copy()
+        for i, k in enumerate(keep):
+            want_c[0, P + i] = c_kv[0, P + k]
+            want_r[0, P + i] = k_rope[0, P + k]
+        assert status[0] == 0 and newp[0] == P + alen, keep
+        assert np.array_equal(ckv2, want_c) and np.array_equal(kr2, want_r), keep
+
+
 # ---------------------------------------------------------------------------
 # Tree build
 # ---------------------------------------------------------------------------
@@ -443,5 +468,6 @@ ALL_PINS = [
     pin_attn_chain_is_causal, pin_attn_decode, pin_attn_tiny_bruteforce, pin_attn_probs,
     pin_attn_prefix_permutation, pin_attn_zero_query, pin_attn_single_key,
     pin_attn_duplicate_keys, pin_accept_golden, pin_accept_properties, pin_compact_golden,
+    pin_compact_closed_forms,
     pin_build_golden, pin_build_bruteforce, pin_build_closed_forms, pin_build_structure,
 ]

@@ -23,6 +23,8 @@ MUTANTS = [
     ("accept skips the first child", "int c = first[cur];", "int c = first[cur] == -1 ? -1 : sib[first[cur]];"),
     ("compaction writes one row late", "memcpy(ckv + (int64_t)(P + i) * ckv_rs",
      "memcpy(ckv + (int64_t)(P + i + (i + 1 < alen)) * ckv_rs"),
+    ("compaction gathers in place (no staging)", ", s_ckv + (size_t)i * DL, sizeof(uint16_t) * DL);",
+     ", ckv + (int64_t)(P + keep[i]) * ckv_rs, sizeof(uint16_t) * DL);"),
     ("depth off by one", "depth[i] = (i == 0) ? 0 : depth[parents[i]] + 1;",
      "depth[i] = (i == 0) ? 1 : depth[parents[i]] + 1;"),
     ("sibling weight keeps the node's own log-prob",
