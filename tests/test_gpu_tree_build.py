@@ -132,3 +132,17 @@ def test_tree_build_weights_that_overflow():
     g = _check(lp, tok, root, 65)
     assert (g["status"] == 0).all() and (g["n_nodes"] == 65).all()
     assert (np.isinf(g["logw"]).sum(axis=1) >= 44).all()
+
+
+def test_tree_build_golden_cases():
+    """The hand-traced trees of the oracle's golden file, bit for bit on the GPU too
+    (all-tied weights, the child-before-sibling insert, running out, a NaN, and the
+    float32 parent-relative sibling weight that decides a tie)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tree_build_cases.json")
+    for case in json.load(open(path))["cases"]:
+        lp = np.array([[[float(x) for x in row] for row in case["lp"]]], dtype=np.float32)
+        tok = np.array([case["tok"]], dtype=np.int32)
+        g = _check(lp, tok, np.array([case["root_token"]], np.int32), case["q_len"])
+        assert g["parents"][0].tolist() == case["parents"], case["name"]

@@ -31,6 +31,9 @@ MUTANTS = [
      "float w = x.logw - L[(size_t)(x.depth - 1) * K + x.rank];", "float w = x.logw;"),
     ("child weight from the node's own depth row", "float w = x.logw + L[(size_t)x.depth * K + 0];",
      "float w = x.logw + L[(size_t)(x.depth - 1) * K + 0];"),
+    ("sibling weight from the parent's weight",
+     "float w = x.logw - L[(size_t)(x.depth - 1) * K + x.rank];\n        w = w + L[(size_t)(x.depth - 1) * K + x.rank + 1];",
+     "float w = lw[x.parent] + L[(size_t)(x.depth - 1) * K + x.rank + 1];"),
     ("ties go to the latest insertion", "if (cand[c].logw > cand[best].logw) best = c;",
      "if (cand[c].logw >= cand[best].logw) best = c;"),
     ("token from rank 0", "ntk[node] = T[(size_t)(x.depth - 1) * K + x.rank];",
