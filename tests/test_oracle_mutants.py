@@ -21,6 +21,7 @@ MUTANTS = [
     ("mask bit order", "word |= (uint64_t)1 << k;", "word |= (uint64_t)1 << (63 - k);"),
     ("accept compares with the wrong target", "if (tok[c] == tgt[cur])", "if (tok[c] == tgt[c])"),
     ("accept skips the first child", "int c = first[cur];", "int c = first[cur] == -1 ? -1 : sib[first[cur]];"),
+    ("walk limit one examination late", "if (examined > Q) {", "if (examined > Q + 1) {"),
     ("compaction writes one row late", "memcpy(ckv + (int64_t)(P + i) * ckv_rs",
      "memcpy(ckv + (int64_t)(P + i + (i + 1 < alen)) * ckv_rs"),
     ("compaction gathers in place (no staging)", ", s_ckv + (size_t)i * DL, sizeof(uint16_t) * DL);",
