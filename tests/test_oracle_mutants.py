@@ -35,6 +35,8 @@ MUTANTS = [
     ("sibling weight from the parent's weight",
      "float w = x.logw - L[(size_t)(x.depth - 1) * K + x.rank];\n        w = w + L[(size_t)(x.depth - 1) * K + x.rank + 1];",
      "float w = lw[x.parent] + L[(size_t)(x.depth - 1) * K + x.rank + 1];"),
+    ("only NaN log-probs rejected", "if (!isfinite(L[e])) st = ORC_BAD_LP;",
+     "if (isnan(L[e])) st = ORC_BAD_LP;"),
     ("ties go to the latest insertion", "if (cand[c].logw > cand[best].logw) best = c;",
      "if (cand[c].logw >= cand[best].logw) best = c;"),
     ("token from rank 0", "ntk[node] = T[(size_t)(x.depth - 1) * K + x.rank];",
