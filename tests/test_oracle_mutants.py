@@ -19,6 +19,11 @@ MUTANTS = [
     ("value from the wrong row", "const uint16_t* vrow = ckv + (int64_t)j * ckv_rs;",
      "const uint16_t* vrow = ckv + (int64_t)(j > 0 ? j - 1 : 0) * ckv_rs;"),
     ("mask bit order", "word |= (uint64_t)1 << k;", "word |= (uint64_t)1 << (63 - k);"),
+    ("parents may point forward", "if (parents[i] < 0 || parents[i] >= i) ok = 0;",
+     "if (parents[i] < 0 || parents[i] >= Q) ok = 0;"),
+    ("last bit of each mask word dropped",
+     "if (a < Q && vis[(size_t)i * Q + a]) word |= (uint64_t)1 << k;",
+     "if (a < Q && k < 63 && vis[(size_t)i * Q + a]) word |= (uint64_t)1 << k;"),
     ("accept compares with the wrong target", "if (tok[c] == tgt[cur])", "if (tok[c] == tgt[c])"),
     ("accept skips the first child", "int c = first[cur];", "int c = first[cur] == -1 ? -1 : sib[first[cur]];"),
     ("walk limit one examination late", "if (examined > Q) {", "if (examined > Q + 1) {"),
