@@ -52,3 +52,30 @@ def test_workload_is_deterministic():
     b = inputs.config(0)
     assert np.array_equal(a.q_lat, b.q_lat) and np.array_equal(a.c_kv, b.c_kv)
     assert a.c_kv.shape == (1, 265, 512) and a.q_lat.shape == (1, 9, 64, 512)
+
+
+def test_draft_batch_rows():
+    """Drafts for the tree build: per (request, depth) row, K finite log-probs of a
+    distribution whose remaining mass sits on the rest of the vocabulary, sorted best
+    first, K distinct tokens; deterministic per seed; the documented top-1 mass."""
+    d = inputs.draft_batch(7, 64, 15, 8)
+    assert d.lp.shape == (64, 15, 8) and d.lp.dtype == np.float32
+    assert d.tok.shape == (64, 15, 8) and d.tok.dtype == np.int32
+    assert np.isfinite(d.lp).all() and (d.lp < 0).all()
+    assert (np.diff(d.lp, axis=2) <= 0).all()
+    head = np.log(np.exp(d.lp.astype(np.float64)).sum(axis=2))
+    assert (head < 0).all()  # the tail keeps some mass
+    assert ((d.tok >= 0) & (d.tok < inputs.VOCAB)).all()
+    assert ((d.root_token >= 0) & (d.root_token < inputs.VOCAB)).all()
+    for b in range(64):
+        for r in range(15):
+            assert len(set(d.tok[b, r].tolist())) == 8
+    assert 0.5 < float(np.exp(d.lp[:, :, 0].astype(np.float64)).mean()) < 0.6
+    again = inputs.draft_batch(7, 64, 15, 8)
+    assert np.array_equal(again.lp, d.lp) and np.array_equal(again.tok, d.tok)
+    other = inputs.draft_batch(8, 64, 15, 8)
+    assert not np.array_equal(other.lp, d.lp)
+    q = inputs.draft_batch(7, 4, 6, 4, quantum=0.5)
+    assert np.array_equal(q.lp, np.round(q.lp * 2) / 2)
+    u = inputs.draft_batch(7, 4, 6, 4, sort=False)
+    assert (np.diff(u.lp, axis=2) > 0).any()
