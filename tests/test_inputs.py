@@ -79,3 +79,12 @@ def test_draft_batch_rows():
     assert np.array_equal(q.lp, np.round(q.lp * 2) / 2)
     u = inputs.draft_batch(7, 4, 6, 4, sort=False)
     assert (np.diff(u.lp, axis=2) > 0).any()
+
+
+def test_draft_trees_have_the_documented_depth():
+    """At budget 32 the drafts give trees of mean depth about 7, some reaching 15
+    (built by the oracle's best-first expansion)."""
+    import oracle
+    d = inputs.draft_batch(7, 64, 15, 8)
+    depth = oracle.tree_build(d.lp, d.tok, d.root_token, 33)["depth"].max(axis=1)
+    assert 6.0 < float(depth.mean()) < 8.5 and int(depth.max()) == 15
