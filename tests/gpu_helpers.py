@@ -17,6 +17,11 @@ MAX_ABS = 2e-2
 REL_L2 = 5e-3
 LSE_MAX_ABS = 5e-3
 
+# Achieved errors of every attention comparison in this session, printed at the
+# end of the run by the terminal summary in conftest.py: (label, max-abs, rel-L2,
+# lse max-abs, rows compared, rows in the output).
+ERROR_LOG: list[tuple] = []
+
 
 def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
@@ -61,10 +66,51 @@ def compare_attention(out_gpu: np.ndarray, ref: np.ndarray, what: str = ""):
     max_abs = float(err.max()) if err.size else 0.0
     denom = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(g - ref) / denom) if denom > 0 else float(np.linalg.norm(g - ref))
+    ERROR_LOG.append((what, max_abs, rel, None, int(g.shape[0]), None))
     assert np.isfinite(g).all(), f"{what}: non-finite output"
     assert max_abs <= MAX_ABS, f"{what}: max abs err {max_abs:.3e} > {MAX_ABS}"
     assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e} > {REL_L2}"
     return max_abs, rel
+
+
+def compare_whole(out: torch.Tensor, lse: torch.Tensor | None, w: inputs.Workload, oracle,
+                  what: str = "", requests_per_chunk: int | None = None):
+    """Every output row of a verify call against the float64 oracle.
+
+    The oracle runs request by request (a chunk of requests at a time, so its
+    float64 output stays a few hundred MB at most).  max-abs is over every
+    element; relative L2 is ||gpu - ref||_2 / ||ref||_2 over the WHOLE output
+    tensor (the sums of squares are accumulated across chunks); lse max-abs is
+    over every row.  Returns (max_abs, rel_l2, lse_max_abs) and records them."""
+    H, DL = w.q_lat.shape[2], w.q_lat.shape[3]
+    rows_per_req = w.q_len * H
+    if requests_per_chunk is None:
+        requests_per_chunk = max(1, (1 << 15) // rows_per_req)
+    flat = out.reshape(-1, DL)
+    lse_flat = None if lse is None else lse.reshape(-1).cpu().numpy().astype(np.float64)
+    max_abs, err2, ref2, lse_err = 0.0, 0.0, 0.0, 0.0
+    for b0 in range(0, w.B, requests_per_chunk):
+        b1 = min(w.B, b0 + requests_per_chunk)
+        rows = np.arange(b0 * rows_per_req, b1 * rows_per_req, dtype=np.int64)
+        o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
+                                        w.parents, w.softmax_scale, rows)
+        g = flat[b0 * rows_per_req:b1 * rows_per_req].float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(g).all(), f"{what}: non-finite output in requests {b0}..{b1 - 1}"
+        d = g - o_ref
+        max_abs = max(max_abs, float(np.abs(d).max()))
+        err2 += float(np.square(d).sum())
+        ref2 += float(np.square(o_ref).sum())
+        if lse_flat is not None:
+            lse_err = max(lse_err, float(np.abs(lse_flat[rows] - l_ref).max()))
+    rel = float(np.sqrt(err2 / ref2)) if ref2 > 0 else float(np.sqrt(err2))
+    total = w.B * rows_per_req
+    ERROR_LOG.append((what, max_abs, rel, lse_err if lse_flat is not None else None, total,
+                      total))
+    assert max_abs <= MAX_ABS, f"{what}: max abs err {max_abs:.3e} > {MAX_ABS}"
+    assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e} > {REL_L2} (whole output)"
+    if lse_flat is not None:
+        assert lse_err <= LSE_MAX_ABS, f"{what}: lse err {lse_err:.3e} > {LSE_MAX_ABS}"
+    return max_abs, rel, lse_err
 
 
 def rows_of(out: torch.Tensor, rows: np.ndarray) -> np.ndarray:
