@@ -106,31 +106,74 @@ def measured_peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def measured_traffic(config_idx: int):
-    """DRAM bytes per verify launch from the committed ncu summary of the default
-    workload, or None when the kernel source changed since that capture."""
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "verify_attn_config2.json")
+
+
+def kernel_source_hash() -> str:
+    """sha256 of the verify kernel's sources (the kernel file and its PTX header)."""
     import hashlib
-    if config_idx != 2:
-        return None
-    path = os.path.join(ROOT, "profiles", "verify_attn_config2.md")
-    try:
-        text = open(path).read()
-    except OSError:
-        return None
-    vals = {}
-    for line in text.splitlines():
-        line = line.strip()
-        for key in ("traffic_bytes_per_launch:", "kernel_source_sha256:"):
-            if line.startswith(key):
-                vals[key] = line.split(":", 1)[1].strip()
     csrc = os.path.join(ROOT, "tree_speculative_decoding_05_b200", "csrc")
     src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("verify_attn.cu", "sm100_ptx.cuh"))
-    if vals.get("kernel_source_sha256:") != hashlib.sha256(src).hexdigest():
+    return hashlib.sha256(src).hexdigest()
+
+
+def measured_traffic(config_idx: int):
+    """DRAM bytes per verify launch of the default workload from the machine-written
+    record of its ncu capture (see record_traffic), or None when there is no record
+    or the kernel source changed since it was taken."""
+    if config_idx != 2:
         return None
     try:
-        return float(vals["traffic_bytes_per_launch:"])
-    except (KeyError, ValueError):
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(rec["traffic_bytes_per_launch"])
+    except (KeyError, TypeError, ValueError):
+        return None
+
+
+_BYTE_UNITS = {"byte": 1.0, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+               "kibyte": 1024.0, "mibyte": 1024.0 ** 2, "gibyte": 1024.0 ** 3}
+
+
+def record_traffic(csv_path: str, command: str) -> int:
+    """Write the traffic record from `ncu -i <capture> --page raw --csv` output of
+    the verify kernel: the mean over the captured launches of
+    dram__bytes_read.sum + dram__bytes_write.sum, with the current source hash."""
+    import csv
+    with open(csv_path, newline="") as f:
+        rows = [r for r in csv.reader(f) if r]
+    head = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    names, units = rows[head], rows[head + 1]
+    col = {n: i for i, n in enumerate(names)}
+    launches = []
+    for r in rows[head + 2:]:
+        if len(r) != len(names) or "verify_attn_kernel" not in r[col["Kernel Name"]]:
+            continue
+        vals = {}
+        for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            scale = _BYTE_UNITS[units[col[m]].strip().lower()]
+            vals[m] = float(r[col[m]].replace(",", "")) * scale
+        launches.append(vals)
+    if not launches:
+        raise SystemExit(f"no verify_attn_kernel launch with DRAM byte counters in {csv_path}")
+    rd = sum(v["dram__bytes_read.sum"] for v in launches) / len(launches)
+    wr = sum(v["dram__bytes_write.sum"] for v in launches) / len(launches)
+    rec = {"kernel": "verify_attn_kernel",
+           "workload": "64 requests x q_len 33 x 64 heads x prefix 4096, bf16 out",
+           "command": command, "launches": len(launches),
+           "dram_bytes_read_per_launch": rd, "dram_bytes_write_per_launch": wr,
+           "traffic_bytes_per_launch": rd + wr,
+           "kernel_source_sha256": kernel_source_hash()}
+    with open(TRAFFIC_RECORD, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
+    return 0
 
 
 class ClockSampler:
@@ -476,6 +519,96 @@ def time_extras(w, d, host, mask, out, lse, workspace, max_prefix, stream, flush
     return res
 
 
+def per_config_report(configs, peaks, device, preloaded=None):
+    """Every workload's calls timed on this run's GPU (the bench line's
+    `per_config`): for each config the inputs are generated and moved to the
+    device, each call runs 5 times untimed, then n calls are captured back to back
+    in one CUDA graph and the replay is timed with CUDA events on the launching
+    stream, median of 5 replays (n = 100, or 20 for calls over 0.5 ms).  When the
+    workload's inputs are under twice the L2, a 256 MB write precedes every call
+    and a graph of the writes alone is timed and subtracted.  Reported: µs per
+    call of build_mask, verify_attn (with its split merge), tree_accept and
+    kv_compact; verify TFLOP/s as a fraction of the burst and the sustained bf16
+    peak; the KV stream's and the compaction's GB/s."""
+    import torch
+
+    from tree_speculative_decoding_05_b200 import ddt
+
+    peak_b = peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)
+    peak_s = peaks.get("bf16_tflops_sustained", peak_b)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for cfg in configs:
+        w = (preloaded or {}).get(cfg) or inputs.config(cfg)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+            torch.bfloat16).to(device)
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+        q_lat, q_rope, c_kv, k_rope = bf(w.q_lat), bf(w.q_rope), bf(w.c_kv), bf(w.k_rope)
+        prefix, parents = i32(w.prefix_lens), i32(w.parents)
+        nt, tt, fc, ns = (i32(w.node_tokens), i32(w.target_tokens), i32(w.next_token),
+                          i32(w.next_sibling))
+        B, Q = w.B, w.q_len
+        max_prefix = int(w.prefix_lens.max())
+        mask, depth, mst = ddt.build_mask(parents)
+        od = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+        out = torch.empty((B, Q, H, DL), dtype=od, device=device)
+        lse = torch.empty((B, Q, H), dtype=torch.float32, device=device) if w.want_lse else None
+        ws, splits = ddt.verify_attn_workspace_size(q_lat, q_rope, c_kv, k_rope, prefix, mask,
+                                                    w.softmax_scale, max_prefix)
+        wsp = torch.empty(ws, dtype=torch.uint8, device=device) if ws else None
+        path = torch.empty((B, Q), dtype=torch.int32, device=device)
+        alen = torch.empty((B,), dtype=torch.int32, device=device)
+        newp = torch.empty((B,), dtype=torch.int32, device=device)
+        vst = torch.empty((B,), dtype=torch.int32, device=device)
+        ddt.tree_accept(nt, tt, fc, ns, path=path, accept_len=alen)
+        input_bytes = sum(t.numel() * t.element_size() for t in (q_lat, q_rope, c_kv, k_rope))
+        fl = flush if input_bytes < 2 * L2_BYTES else None
+        calls = {
+            "build_mask": lambda: ddt.build_mask(parents, mask=mask, depth=depth, status=mst),
+            "verify_attn": lambda: ddt.verify_attn(q_lat, q_rope, c_kv, k_rope, prefix, mask,
+                                                   w.softmax_scale, max_prefix=max_prefix,
+                                                   out=out, lse=lse, workspace=wsp,
+                                                   status=vst),
+            "tree_accept": lambda: ddt.tree_accept(nt, tt, fc, ns, path=path, accept_len=alen),
+            "kv_compact": lambda: ddt.kv_compact(c_kv, k_rope, prefix, path, alen,
+                                                 new_prefix_lens=newp),
+        }
+        us = {}
+        for name, fn in calls.items():
+            for _ in range(5):
+                fn()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            n = 20 if time.perf_counter() - t0 > 0.5e-3 else 100
+            us[name] = graph_time_us(fn, n, fl, reps=5)
+        torch.cuda.synchronize()
+        path_h, alen_h = path.cpu().numpy(), alen.cpu().numpy()
+        moved = sum(int((path_h[b, :alen_h[b]] != np.arange(alen_h[b])).sum()) for b in range(B))
+        flops = verify_flops(w.prefix_lens, w.parents)
+        tflops = flops / (us["verify_attn"] * 1e-6) / 1e12
+        res[str(cfg)] = {
+            "workload": w.name, "B": B, "q_len": Q, "prefix_max": max_prefix,
+            "out": w.out_dtype, "lse": bool(w.want_lse), "kv_splits": splits,
+            "calls_us": us,
+            "verify_gflop": flops / 1e9,
+            "verify_tflops": tflops,
+            "verify_frac_burst": tflops / peak_b,
+            "verify_frac_sustained": tflops / peak_s,
+            "kv_stream_gbs": float((w.prefix_lens.astype(np.float64) + Q).sum()) * (DL + DR) * 2
+                             / (us["verify_attn"] * 1e-6) / 1e9,
+            "kv_compact_rows_moved": moved,
+            "kv_compact_gbs": 2.0 * moved * (DL + DR) * 2 / (us["kv_compact"] * 1e-6) / 1e9,
+            "statuses_ok": bool((vst.cpu().numpy() == 0).all() and (mst.cpu().numpy() == 0).all()),
+            "l2": "flushed before every call (flush subtracted)" if fl is not None
+                  else "inputs over twice the L2: no flush",
+        }
+        del q_lat, q_rope, c_kv, k_rope, out, lse, wsp, calls
+        torch.cuda.empty_cache()
+    return res
+
+
 def per_call_report(args) -> int:
     """Every call of the path timed alone per workload: 10 warm-up calls, then 100
     calls captured back to back in a CUDA graph and the replay timed with events,
@@ -687,6 +820,14 @@ def main(argv=None) -> int:
                     help="with several GPUs: every rank runs its own batch of the workload "
                          "(replicas, weak scaling) or the ranks split one batch by request "
                          "with the longest-first rule (strong scaling)")
+    ap.add_argument("--record-traffic", metavar="RAW_CSV",
+                    help="write the verify kernel's DRAM traffic record (profiles/"
+                         "verify_attn_config2.json) from `ncu -i <capture> --page raw --csv` "
+                         "output; no GPU needed")
+    ap.add_argument("--capture-command", default="",
+                    help="with --record-traffic: the ncu command that made the capture")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-call timings of all five workloads")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the timings of the calls outside the step (tree build, fused "
                          "accept+compaction, chained decode step)")
@@ -696,6 +837,8 @@ def main(argv=None) -> int:
 
     world, rank, local = dist_env()
 
+    if args.record_traffic:
+        return record_traffic(args.record_traffic, args.capture_command)
     if args.per_call:
         return per_call_report(args)
     if args.accept_sweep:
@@ -904,6 +1047,12 @@ def main(argv=None) -> int:
         extras = time_extras(w, d, host, mask, out, lse, workspace if ws_bytes else None,
                              max_prefix, stream, flush, max(args.steps, 20), args.warmup)
 
+    # ---- the other workloads' calls, graph-timed on this GPU ---------------
+    per_config = None
+    if rank == 0 and world == 1 and not args.no_per_config:
+        per_config = per_config_report([0, 1, 2, 3, 4], measured_peaks()[0], device,
+                                       preloaded={args.config: w})
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1) -------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -956,6 +1105,7 @@ def main(argv=None) -> int:
                          "algorithmic_bytes": bytes_local,
                          "kernel": "verify_attn_kernel"},
             "extras": extras,
+            "per_config": per_config,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,

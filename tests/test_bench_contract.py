@@ -31,3 +31,30 @@ def test_reference_arm_prints_the_contract_line():
 def test_too_few_warmup_steps_are_refused():
     r = _run("--impl", "reference", "--steps", "1", "--warmup", "2", "--config", "0")
     assert r.returncode != 0
+
+
+def test_traffic_record_from_ncu_raw_csv(tmp_path, monkeypatch):
+    """--record-traffic reads ncu's raw CSV page (a header row of metric names, a
+    row of units, one row per launch) and writes the mean DRAM bytes per verify
+    launch with the kernel source hash; measured_traffic reads it back only while
+    the hash matches."""
+    sys.path.insert(0, ROOT)
+    import bench
+    csv_path = tmp_path / "raw.csv"
+    csv_path.write_text(
+        '"ID","Kernel Name","dram__bytes_read.sum","dram__bytes_write.sum"\n'
+        '"","","Mbyte","Gbyte"\n'
+        '"0","ddt::build_mask_kernel(const int *)","1.00","0.001"\n'
+        '"1","ddt::verify_attn_kernel(CUtensorMap_st, ddt::VerifyParams)","460.00","0.1187"\n'
+        '"2","ddt::verify_attn_kernel(CUtensorMap_st, ddt::VerifyParams)","462.00","0.1189"\n')
+    rec_path = tmp_path / "rec.json"
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(rec_path))
+    assert bench.record_traffic(str(csv_path), "ncu ...") == 0
+    rec = json.loads(rec_path.read_text())
+    assert rec["launches"] == 2
+    assert abs(rec["traffic_bytes_per_launch"] - (461.0e6 + 118.8e6)) < 1.0
+    assert bench.measured_traffic(2) == rec["traffic_bytes_per_launch"]
+    assert bench.measured_traffic(3) is None
+    rec["kernel_source_sha256"] = "0" * 64
+    rec_path.write_text(json.dumps(rec))
+    assert bench.measured_traffic(2) is None
