@@ -22,9 +22,13 @@
  *                      Under Time Pressure"
  *
  * Conventions shared by every call
- *   - Every pointer argument is a DEVICE pointer owned by the caller.  The
- *     library never allocates or frees device memory; scratch space that a call
- *     needs is passed in by the caller (see ddt_verify_attn_workspace_size).
+ *   - Every pointer argument is a DEVICE pointer owned by the caller.  No call
+ *     allocates or frees device memory; scratch space that a call needs is
+ *     passed in by the caller (see ddt_verify_attn_workspace_size).  One
+ *     exception in footprint, not in calls: loading the library's device code
+ *     on a GPU reserves the 32 MiB static scratch array of
+ *     ddt_verify_attn_noalloc there until the process exits, whether or not
+ *     that entry point is ever called.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronises the host.
  *   - Arguments that the host can check (sizes, null pointers, alignment,
@@ -245,9 +249,11 @@ DDT_API ddt_status ddt_verify_attn(const ddt_attn_args* args, ddt_stream_t strea
  * fixed scratch array inside the library (ddt_verify_attn_noalloc_scratch_bytes()
  * bytes, 32 MiB, held on every GPU that loads the library until the process
  * exits).  It allocates nothing.
- *   - The first call on a device looks the array's address up (this may load
- *     the library's device code on that device); make it before any stream
- *     capture on that device.
+ *   - The first call in a CUDA context (normally the device's primary
+ *     context) looks the array's address up (this may load the library's
+ *     device code on that device); make it before any stream capture on that
+ *     device.  The address is remembered per context (by the driver's unique
+ *     context ID), so a reset or replaced context gets a fresh lookup.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents; nothing in it needs to start at zero.  Calls that overlap on
  *     the GPU race on it: order them (one stream, or events).

@@ -13,7 +13,9 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import DeviceWorkload, LSE_MAX_ABS, MAX_ABS, REL_L2
+import oracle
+from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, MAX_ABS, REL_L2, compare_attention,
+                         rows_of, sample_rows)
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -62,6 +64,69 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         torch.cuda.synchronize()
         _close(out, ref_out, MAX_ABS, REL_L2)
         _close(lse, ref_lse, LSE_MAX_ABS)
+        _check_oracle(out, lse, w, f"no-alloc call {call}")
+    assert ddt.fault_flags(reset=True) == 0
+
+
+def _check_oracle(out, lse, w, what):
+    """Sampled rows (and the last node of every request) against the float64 oracle."""
+    H = 64
+    must = np.concatenate([np.arange((b + 1) * w.q_len * H - H, (b + 1) * w.q_len * H)
+                           for b in range(w.B)])
+    rows = sample_rows(w.B, w.q_len, H, 768, seed=w.seed, must=must)
+    o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
+                                    w.parents, w.softmax_scale, rows)
+    compare_attention(rows_of(out, rows), o_ref, what)
+    assert np.abs(lse.reshape(-1).cpu().numpy()[rows] - l_ref).max() <= LSE_MAX_ABS, what
+
+
+def _auto_plan(lib, a):
+    """The split count the automatic plan picks, and the one the no-alloc call is
+    documented to use: the largest count below the plan whose partials fit the
+    scratch array, else one split (which needs none)."""
+    cap = int(lib.ddt_verify_attn_noalloc_scratch_bytes())
+    planned = int(lib.ddt_verify_attn_num_splits(ctypes.byref(a)))
+    if int(lib.ddt_verify_attn_workspace_size(ctypes.byref(a))) <= cap:
+        return planned, planned
+    for s in range(planned - 1, 1, -1):
+        a.num_splits = s
+        fits = int(lib.ddt_verify_attn_workspace_size(ctypes.byref(a))) <= cap
+        a.num_splits = 0
+        if fits:
+            return planned, s
+    return planned, 1
+
+
+@pytest.mark.parametrize("B,Q,P,want", [(3, 33, 20000, 2), (4, 128, 32768, 1)])
+def test_noalloc_automatic_plan_larger_than_its_scratch(B, Q, P, want):
+    """num_splits = 0 on shapes whose planned partials exceed the 32 MiB array:
+    3 x q_len 33 x prefix 20000 plans 4 splits (50 MB of partials) and must step
+    down to 2 (25 MB); 4 x q_len 128 x prefix 32768 plans 2 splits (134 MB) and
+    must fall back to one split.  The result equals ddt_verify_attn forced to
+    that split count bit for bit, and the oracle within the tolerances."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = _noalloc_lib()
+    w = inputs.make_workload("noalloc-auto", 5150 + Q, B, Q, [P] * B, want_lse=True)
+    dw = DeviceWorkload(w)
+    mask, _, _ = ddt.build_mask(dw.parents)
+    out = torch.full((B, Q, 64, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Q, 64), float("nan"), dtype=torch.float32, device="cuda")
+    a = ddt._attn_args(dw.q_lat, dw.q_rope, dw.c_kv, dw.k_rope, dw.prefix, mask,
+                       w.softmax_scale, out, lse, P, 0, None, None)
+    planned, used = _auto_plan(lib, a)
+    assert used == want and planned > used
+    assert int(lib.ddt_verify_attn_workspace_size(ctypes.byref(a))) > \
+        int(lib.ddt_verify_attn_noalloc_scratch_bytes())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.ddt_verify_attn_noalloc(ctypes.byref(a), stream) == ddt.DDT_OK
+    torch.cuda.synchronize()
+    ref_out, ref_lse = ddt.verify_attn(dw.q_lat, dw.q_rope, dw.c_kv, dw.k_rope, dw.prefix, mask,
+                                       w.softmax_scale, max_prefix=P, want_lse=True,
+                                       num_splits=used)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    _check_oracle(out, lse, w, f"no-alloc automatic B={B} Q={Q} P={P}")
     assert ddt.fault_flags(reset=True) == 0
 
 

@@ -13,9 +13,13 @@
 //   * The array is a file-scope static device array of kScratchBytes (32 MiB).
 //     Every GPU on which the library's device code is loaded holds it until the
 //     process exits.
-//   * The first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress, which may load the library's device code on that
-//     device); make that first call before any stream capture on the device.
+//   * The first call in a CUDA context (normally a device's primary context)
+//     looks up the array's device address there (cudaGetSymbolAddress, which
+//     may load the library's device code on that device); make that first call
+//     before any stream capture on the device.  The address is remembered per
+//     context, keyed by the driver's unique context ID, so a context that is
+//     reset (cudaDeviceReset) or replaced gets a fresh lookup instead of a
+//     stale address.
 //   * All calls on a device share the one array, and it keeps whatever the last
 //     call left in it.  Nothing in it needs to start at zero: every split
 //     writes all of its partial rows before the merge reads them, and empty
@@ -27,6 +31,7 @@
 //     whose partials exceed the array is rejected with DDT_ERR_UNSUPPORTED
 //     before anything is launched.
 //   * It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -38,27 +43,76 @@
 namespace {
 
 constexpr size_t kScratchBytes = static_cast<size_t>(32) << 20;
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 static __device__ __align__(256) unsigned char g_verify_scratch[kScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (looked up once per
-// device, with that device current).
-ddt_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DDT_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return DDT_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+struct DriverFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+const DriverFns& driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || p == nullptr)
-      return DDT_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return fns;
+}
+
+// Unique ID of the calling thread's current context (0 if there is none or the
+// driver cannot say).  IDs are never reused within a process.
+unsigned long long current_context_id() {
+  const DriverFns& f = driver_fns();
+  if (!f.get_current || !f.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+std::mutex g_scratch_mu;
+unsigned long long g_ctx_id[kMaxContexts] = {};
+void* g_ctx_ptr[kMaxContexts] = {};
+int g_ctx_next = 0;
+
+// Device address of the scratch array in the current context: looked up with
+// cudaGetSymbolAddress once per context and remembered under the context's
+// unique ID.  Without a usable ID (no current context yet, or a driver that
+// cannot report one) the address is looked up again on every call.
+ddt_status scratch_address(void** out) {
+  unsigned long long id = current_context_id();
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (id != 0) {
+    for (int i = 0; i < kMaxContexts; ++i)
+      if (g_ctx_id[i] == id) {
+        *out = g_ctx_ptr[i];
+        return DDT_OK;
+      }
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || p == nullptr)
+    return DDT_ERR_CUDA;
+  if (id == 0) id = current_context_id();  // the lookup may have made the context current
+  if (id != 0) {
+    g_ctx_id[g_ctx_next] = id;
+    g_ctx_ptr[g_ctx_next] = p;
+    g_ctx_next = (g_ctx_next + 1) % kMaxContexts;
+  }
+  *out = p;
   return DDT_OK;
 }
 
