@@ -7,19 +7,40 @@ import torch
 
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
-# Tolerances for the attention output against the float64 oracle.  The weights
-# enter P V as bf16 (rounding to nearest: relative error <= 2^-8 each, largely
-# averaging out over many keys), and a bf16 output rounds once more (at most half
-# an ulp: 0.0156 for |o| in [4, 8)), so max-abs 2e-2 covers outputs up to |o| ~ 8
-# with the weights' error on top; the relative L2 bound 5e-3 and the lse bound
-# 5e-3 express the same budget in those measures.
+# Tolerances for the attention output against the float64 oracle.  MAX_ABS bounds
+# the error of the computation: the weights enter P V as bf16 (rounding to
+# nearest: relative error <= 2^-8 each, largely averaging out over many keys) and
+# everything else accumulates in fp32.  The output's own rounding to its dtype is
+# allowed on top, elementwise: half an ulp of the output dtype at the exact value
+# (bf16: 0.0156 for |o| in [4, 8), 0.03125 for |o| in [8, 16)).  No output in that
+# dtype can be closer to the exact value than that, and the row-scaled workload
+# (cache rows N(0,1) x U(0.5, 2)) has outputs above 8, where a literal 2e-2 bound
+# on a bf16 value cannot be met.  The relative L2 bound 5e-3 (over the whole
+# compared tensor) and the lse bound 5e-3 take no such allowance.
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
 LSE_MAX_ABS = 5e-3
 
+
+def out_format(t: torch.Tensor) -> str:
+    """Output dtype of a verify call's result: "bf16" or "f32"."""
+    return "bf16" if t.dtype == torch.bfloat16 else "f32"
+
+
+def half_ulp(ref: np.ndarray, fmt: str) -> np.ndarray:
+    """Half a unit in the last place of the output dtype at |ref| (the largest
+    error of a round-to-nearest conversion of ref to that dtype): bf16 keeps 8
+    significant bits, fp32 24; magnitudes below the smallest normal use its ulp."""
+    bits = 8 if fmt == "bf16" else 24
+    _, ex = np.frexp(np.abs(ref))            # |ref| = m * 2^ex, m in [0.5, 1)
+    ex = np.maximum(ex, -125)                # fp32/bf16 smallest normal: 2^-126
+    return np.ldexp(1.0, ex - bits - 1)
+
+
 # Achieved errors of every attention comparison in this session, printed at the
 # end of the run by the terminal summary in conftest.py: (label, max-abs, rel-L2,
-# lse max-abs, rows compared, rows in the output).
+# lse max-abs, rows compared, rows in the output, largest error beyond the
+# output's own rounding).
 ERROR_LOG: list[tuple] = []
 
 
@@ -59,16 +80,21 @@ class DeviceWorkload:
         return out, lse, status
 
 
-def compare_attention(out_gpu: np.ndarray, ref: np.ndarray, what: str = ""):
-    """Max-abs and relative-L2 error of a GPU result against float64 values."""
+def compare_attention(out_gpu: np.ndarray, ref: np.ndarray, what: str = "", *, fmt: str):
+    """Errors of a GPU result (values of output dtype `fmt`) against float64
+    values: max-abs, relative L2 over the compared rows, and the largest error
+    beyond the output's own rounding (|gpu - ref| - half_ulp(ref)), which must
+    stay within MAX_ABS."""
     g = out_gpu.astype(np.float64)
     err = np.abs(g - ref)
     max_abs = float(err.max()) if err.size else 0.0
+    excess = float((err - half_ulp(ref, fmt)).max()) if err.size else 0.0
     denom = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(g - ref) / denom) if denom > 0 else float(np.linalg.norm(g - ref))
-    ERROR_LOG.append((what, max_abs, rel, None, int(g.shape[0]), None))
+    ERROR_LOG.append((what, max_abs, rel, None, int(g.shape[0]), None, excess))
     assert np.isfinite(g).all(), f"{what}: non-finite output"
-    assert max_abs <= MAX_ABS, f"{what}: max abs err {max_abs:.3e} > {MAX_ABS}"
+    assert excess <= MAX_ABS, (f"{what}: error beyond the output's rounding {excess:.3e} > "
+                               f"{MAX_ABS} (max abs {max_abs:.3e})")
     assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e} > {REL_L2}"
     return max_abs, rel
 
@@ -78,17 +104,20 @@ def compare_whole(out: torch.Tensor, lse: torch.Tensor | None, w: inputs.Workloa
     """Every output row of a verify call against the float64 oracle.
 
     The oracle runs request by request (a chunk of requests at a time, so its
-    float64 output stays a few hundred MB at most).  max-abs is over every
-    element; relative L2 is ||gpu - ref||_2 / ||ref||_2 over the WHOLE output
-    tensor (the sums of squares are accumulated across chunks); lse max-abs is
-    over every row.  Returns (max_abs, rel_l2, lse_max_abs) and records them."""
+    float64 output stays a few hundred MB at most).  max-abs and the error beyond
+    the output's own rounding are over every element (the latter must stay
+    within MAX_ABS); relative L2 is ||gpu - ref||_2 / ||ref||_2 over the WHOLE
+    output tensor (the sums of squares are accumulated across chunks); lse
+    max-abs is over every row.  Returns (max_abs, rel_l2, lse_max_abs) and
+    records them."""
     H, DL = w.q_lat.shape[2], w.q_lat.shape[3]
     rows_per_req = w.q_len * H
     if requests_per_chunk is None:
         requests_per_chunk = max(1, (1 << 15) // rows_per_req)
+    fmt = out_format(out)
     flat = out.reshape(-1, DL)
     lse_flat = None if lse is None else lse.reshape(-1).cpu().numpy().astype(np.float64)
-    max_abs, err2, ref2, lse_err = 0.0, 0.0, 0.0, 0.0
+    max_abs, err2, ref2, lse_err, excess = 0.0, 0.0, 0.0, 0.0, -np.inf
     for b0 in range(0, w.B, requests_per_chunk):
         b1 = min(w.B, b0 + requests_per_chunk)
         rows = np.arange(b0 * rows_per_req, b1 * rows_per_req, dtype=np.int64)
@@ -98,6 +127,7 @@ def compare_whole(out: torch.Tensor, lse: torch.Tensor | None, w: inputs.Workloa
         assert np.isfinite(g).all(), f"{what}: non-finite output in requests {b0}..{b1 - 1}"
         d = g - o_ref
         max_abs = max(max_abs, float(np.abs(d).max()))
+        excess = max(excess, float((np.abs(d) - half_ulp(o_ref, fmt)).max()))
         err2 += float(np.square(d).sum())
         ref2 += float(np.square(o_ref).sum())
         if lse_flat is not None:
@@ -105,8 +135,9 @@ def compare_whole(out: torch.Tensor, lse: torch.Tensor | None, w: inputs.Workloa
     rel = float(np.sqrt(err2 / ref2)) if ref2 > 0 else float(np.sqrt(err2))
     total = w.B * rows_per_req
     ERROR_LOG.append((what, max_abs, rel, lse_err if lse_flat is not None else None, total,
-                      total))
-    assert max_abs <= MAX_ABS, f"{what}: max abs err {max_abs:.3e} > {MAX_ABS}"
+                      total, excess))
+    assert excess <= MAX_ABS, (f"{what}: error beyond the output's rounding {excess:.3e} > "
+                               f"{MAX_ABS} (max abs {max_abs:.3e})")
     assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e} > {REL_L2} (whole output)"
     if lse_flat is not None:
         assert lse_err <= LSE_MAX_ABS, f"{what}: lse err {lse_err:.3e} > {LSE_MAX_ABS}"

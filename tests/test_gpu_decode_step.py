@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import MAX_ABS, REL_L2, bf16_tensor, compare_attention, i32
+from gpu_helpers import MAX_ABS, REL_L2, bf16_tensor, compare_attention, i32, out_format
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -123,7 +123,8 @@ def _compare(chain, ref, c_ref, k_ref, P_ref, root_ref):
         assert (bufs["status"].cpu().numpy() == 0).all()
         assert (bufs["verify_status"].cpu().numpy() == 0).all()
         compare_attention(bufs["out"].float().cpu().numpy().reshape(-1, DL),
-                          r["out"].reshape(-1, DL), "decode-step attention")
+                          r["out"].reshape(-1, DL), "decode-step attention",
+                          fmt=out_format(bufs["out"]))
         assert np.array_equal(bufs["path"].cpu().numpy(), r["path"])
         assert np.array_equal(bufs["accept_len"].cpu().numpy(), r["alen"])
     s = chain.state

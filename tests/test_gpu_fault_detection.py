@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import DeviceWorkload, compare_attention
+from gpu_helpers import DeviceWorkload, compare_attention, out_format
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -33,7 +33,7 @@ def test_bounded_wait_gives_up_and_the_context_survives():
     o_ref, _ = oracle.attn_all(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens, w.parents,
                                w.softmax_scale)
     compare_attention(out.float().cpu().numpy().reshape(-1, 512), o_ref.reshape(-1, 512),
-                      "after the self-test")
+                      "after the self-test", fmt=out_format(out))
     assert ddt.fault_flags(reset=True) == 0
 
 

@@ -13,7 +13,7 @@ import torch
 import oracle
 import oracle_pins
 from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, compare_attention, compare_whole, i32,
-                         rows_of, sample_rows)
+                         out_format, rows_of, sample_rows)
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -178,7 +178,7 @@ def _check_attention(dw: DeviceWorkload, rows=None, num_splits=0, out_dtype=None
         rows = np.arange(w.B * w.q_len * H, dtype=np.int64)
     o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
                                     w.parents, w.softmax_scale, rows)
-    compare_attention(rows_of(out, rows), o_ref, what)
+    compare_attention(rows_of(out, rows), o_ref, what, fmt=out_format(out))
     l_gpu = lse.reshape(-1).cpu().numpy()[rows].astype(np.float64)
     assert np.max(np.abs(l_gpu - l_ref)) <= LSE_MAX_ABS, what
     return out, lse
@@ -297,7 +297,7 @@ def test_verify_attn_random_shapes(seed):
     torch.cuda.synchronize()
     o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
                                     w.parents, w.softmax_scale, rows)
-    compare_attention(rows_of(out, rows), o_ref, what + " split")
+    compare_attention(rows_of(out, rows), o_ref, what + " split", fmt=out_format(out))
     assert np.abs(lse.reshape(-1).cpu().numpy()[rows] - l_ref).max() <= LSE_MAX_ABS, what
 
 

@@ -11,8 +11,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, MAX_ABS, compare_attention, rows_of,
-                         sample_rows)
+from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, MAX_ABS, compare_attention, out_format,
+                         rows_of, sample_rows)
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -40,7 +40,7 @@ def _check(w, rows=None, num_splits=0, what=""):
         rows = np.arange(w.B * w.q_len * H, dtype=np.int64)
     o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
                                     w.parents, w.softmax_scale, rows)
-    compare_attention(rows_of(out, rows), o_ref, what)
+    compare_attention(rows_of(out, rows), o_ref, what, fmt=out_format(out))
     l_gpu = lse.reshape(-1).cpu().numpy()[rows].astype(np.float64)
     assert np.max(np.abs(l_gpu - l_ref)) <= LSE_MAX_ABS, what
     # and against the fused pass: both are within MAX_ABS of the exact values, so

@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import DeviceWorkload, LSE_MAX_ABS, bf16_tensor, compare_attention, i32
+from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, bf16_tensor, compare_attention, i32,
+                         out_format)
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +49,8 @@ def test_verify_on_interleaved_cache(split_tail):
     rows = np.arange(w.B * w.q_len * 64, dtype=np.int64)
     o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
                                     w.parents, w.softmax_scale, rows)
-    compare_attention(out.float().cpu().numpy().reshape(-1, 512), o_ref, "interleaved cache")
+    compare_attention(out.float().cpu().numpy().reshape(-1, 512), o_ref, "interleaved cache",
+                      fmt=out_format(out))
     assert np.abs(lse.reshape(-1).cpu().numpy() - l_ref).max() <= LSE_MAX_ABS
 
 

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from gpu_helpers import (DeviceWorkload, LSE_MAX_ABS, MAX_ABS, REL_L2, compare_attention,
-                         rows_of, sample_rows)
+                         out_format, rows_of, sample_rows)
 from tree_speculative_decoding_05_b200 import ddt, inputs
 
 pytestmark = pytest.mark.gpu
@@ -76,7 +76,7 @@ def _check_oracle(out, lse, w, what):
     rows = sample_rows(w.B, w.q_len, H, 768, seed=w.seed, must=must)
     o_ref, l_ref = oracle.attn_rows(w.q_lat, w.q_rope, w.c_kv, w.k_rope, w.prefix_lens,
                                     w.parents, w.softmax_scale, rows)
-    compare_attention(rows_of(out, rows), o_ref, what)
+    compare_attention(rows_of(out, rows), o_ref, what, fmt=out_format(out))
     assert np.abs(lse.reshape(-1).cpu().numpy()[rows] - l_ref).max() <= LSE_MAX_ABS, what
 
 
