@@ -17,9 +17,8 @@ SRC = os.path.join(build.CSRC, "verify_attn.cu")
 CASES = [
     ("-DDDT_VERIFY_K_STAGE_CHUNKS=1 -DDDT_VERIFY_V_KEYS=32", True),   # the earlier layout
     ("-DDDT_VERIFY_TILE_KEYS=256", True),                            # wide tiles
-    ("-DDDT_VERIFY_QK_ISSUERS=3 -DDDT_VERIFY_K_STAGE_CHUNKS=1 -DDDT_VERIFY_K_STAGES=3 "
-     "-DDDT_VERIFY_V_STAGES=2", True),                               # three S issuers
-    ("-DDDT_VERIFY_QK_ISSUERS=3", False),                            # 3 rings x 2 x 16 KB: too big
+    ("-DDDT_VERIFY_WARP_MAP=10", True),                              # no idle warp
+    ("-DDDT_VERIFY_K_STAGES=3", False),                              # 2 rings x 3 x 16 KB: too big
 ]
 
 

@@ -146,16 +146,39 @@ __global__ void __launch_bounds__(kAcceptWarps * 32) tree_accept_kernel(
 // Compaction.  [Race Conditions] "The Cache Compaction Problem": row P+i takes
 // old row P+keep[i].  A parallel in-place gather races when keep[j] = i' (row
 // i' read by one thread while another writes it); the pages route the gather
-// through scratch buffers.  Here one CTA owns a request: it reads every kept row
-// (latent and rope parts) into shared memory with 16-byte loads, synchronises,
-// and only then writes, so no write can precede a read of the same row — for
-// any path, without scratch memory.  Rows that do not move (keep[i] == i) are
-// not rewritten.
+// through scratch buffers.  Here a write can only clobber the same bytes of a
+// row that some index reads, and a row's column ranges never alias, so each
+// row (latent then rope, 72 vectors of 16 bytes) is cut into kCompactSlices
+// column slices of kSliceVec vectors and one CTA owns one slice of one request:
+// it reads that slice of every moving row into shared memory, synchronises, and
+// only then writes it.  No write precedes a read of the same bytes, for any
+// path, without scratch memory.  The slices of a request are one thread-block
+// cluster; a cluster barrier after every CTA has read the request's prefix
+// length lets the first slice publish the new prefix length even when
+// new_prefix_lens aliases prefix_lens.  A slice stages at most 128 x 288 bytes
+// (36 KB), so several CTAs share an SM and one request's reads overlap
+// another's writes.  Rows that do not move (keep[i] == i) are not rewritten.
 // ---------------------------------------------------------------------------
-constexpr int kCompactThreads = 256;
+#ifndef DDT_COMPACT_THREADS
+#define DDT_COMPACT_THREADS 256
+#endif
+#ifndef DDT_COMPACT_SLICES
+#define DDT_COMPACT_SLICES 4
+#endif
+constexpr int kCompactThreads = DDT_COMPACT_THREADS;
 constexpr int kLatVec = DDT_D_LATENT * 2 / 16;  // 16-byte vectors per latent row (64)
 constexpr int kRopeVec = DDT_D_ROPE * 2 / 16;   // per rope row (8)
 constexpr int kRowVec = kLatVec + kRopeVec;
+constexpr int kCompactSlices = DDT_COMPACT_SLICES;  // a cluster: at most 8
+constexpr int kSliceVec = kRowVec / kCompactSlices;  // 4 slices: 18 vectors = 288 bytes
+static_assert(kSliceVec * kCompactSlices == kRowVec, "row slices cover the row");
+static_assert(kSliceVec % 2 == 0, "a slice is whole 32-byte sectors");
+static_assert(kCompactSlices <= 8, "the slices of a request form one portable cluster");
+
+__device__ __forceinline__ void compact_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // Asynchronous 16-byte copy global -> shared (cp.async, L2 only): a thread can have
 // all of its copies in flight at once instead of one load per loop iteration.
@@ -168,19 +191,22 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// Moves rows P+keep[i] -> P+i (i < alen) of request b, both caches, through
-// shared memory: every moving row is read before any is written.  Called by all
-// kCompactThreads threads of the CTA; s_rows holds alen * kRowVec vectors.
+// Moves slice `slice` (row vectors [slice * kSliceVec, + kSliceVec)) of rows
+// P+keep[i] -> P+i (i < alen) of request b, both caches, through shared memory:
+// the slice of every moving row is read before any is written.  Called by all
+// kCompactThreads threads of the CTA; s_rows holds alen * kSliceVec vectors.
 __device__ void compact_rows(uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope,
                              int64_t ckv_bs, int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs, int b,
-                             int P, int alen, const int32_t* s_keep, uint4* s_rows) {
+                             int P, int alen, const int32_t* s_keep, uint4* s_rows, int slice) {
   const uint4* ckv_b = reinterpret_cast<const uint4*>(c_kv + b * ckv_bs);
   const uint4* kr_b = reinterpret_cast<const uint4*>(k_rope + b * kr_bs);
   const int64_t ckv_rv = ckv_rs / 8, kr_rv = kr_rs / 8;  // row strides in 16-byte vectors
-  const int total = alen * kRowVec;
-  // Phase 1: every moving row into shared memory, all copies in flight together.
+  const int total = alen * kSliceVec;
+  const int v0 = slice * kSliceVec;
+  // Phase 1: the slice of every moving row into shared memory, all copies in
+  // flight together.
   for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
-    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    const int i = idx / kSliceVec, v = v0 + (idx - i * kSliceVec);
     if (s_keep[i] == i) continue;
     const int64_t src_row = P + s_keep[i];
     cp_async16(&s_rows[idx], (v < kLatVec) ? ckv_b + (src_row * ckv_rv + v)
@@ -188,11 +214,11 @@ __device__ void compact_rows(uint16_t* __restrict__ c_kv, uint16_t* __restrict__
   }
   cp_async_wait_all();
   __syncthreads();
-  // Phase 2: write rows P .. P+alen-1 (only those that move).
+  // Phase 2: write the slice of rows P .. P+alen-1 (only those that move).
   uint4* ckv_w = reinterpret_cast<uint4*>(c_kv + b * ckv_bs);
   uint4* kr_w = reinterpret_cast<uint4*>(k_rope + b * kr_bs);
   for (int idx = threadIdx.x; idx < total; idx += kCompactThreads) {
-    const int i = idx / kRowVec, v = idx - i * kRowVec;
+    const int i = idx / kSliceVec, v = v0 + (idx - i * kSliceVec);
     if (s_keep[i] == i) continue;
     const int64_t dst_row = P + i;
     if (v < kLatVec) ckv_w[dst_row * ckv_rv + v] = s_rows[idx];
@@ -200,17 +226,23 @@ __device__ void compact_rows(uint16_t* __restrict__ c_kv, uint16_t* __restrict__
   }
 }
 
-__global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
-    uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
-    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* prefix_lens,
-    const int32_t* __restrict__ path, const int32_t* __restrict__ accept_len, int q_len,
-    int32_t* new_prefix_lens, int32_t* __restrict__ status) {
-  extern __shared__ uint4 s_rows[];  // [alen][kRowVec]
+// Grid: kCompactSlices CTAs (one cluster) per request, CTA b * kCompactSlices + s
+// moving slice s of request b.
+__global__ void __cluster_dims__(kCompactSlices, 1, 1) __launch_bounds__(kCompactThreads)
+    kv_compact_kernel(uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs,
+                      int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs, int capacity,
+                      const int32_t* prefix_lens, const int32_t* __restrict__ path,
+                      const int32_t* __restrict__ accept_len, int q_len, int32_t* new_prefix_lens,
+                      int32_t* __restrict__ status) {
+  extern __shared__ uint4 s_rows[];  // [alen][kSliceVec]
   __shared__ int32_t s_keep[DDT_MAX_Q_LEN];
   __shared__ int s_state;  // 0 ok, else status code
-  const int b = blockIdx.x;
-  const int P = prefix_lens[b];  // read by every thread before the first barrier, so
-  const int alen = accept_len[b];  // new_prefix_lens may be prefix_lens itself
+  const int b = blockIdx.x / kCompactSlices;
+  const int slice = blockIdx.x % kCompactSlices;
+  // Read by every thread of every slice before the cluster barrier below, so
+  // new_prefix_lens may be prefix_lens itself.
+  const int P = prefix_lens[b];
+  const int alen = accept_len[b];
   if (threadIdx.x == 0) {
     int st = DDT_REQ_OK;
     if (alen < 1 || alen > q_len) st = DDT_REQ_BAD_LENGTH;
@@ -229,15 +261,17 @@ __global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
     __syncthreads();
   }
   const int st = s_state;
+  // Every slice has read P (and the same path, so the same verdict).
+  compact_cluster_sync();
   if (st != DDT_REQ_OK) {
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && slice == 0) {
       if (status) status[b] = st;
       if (new_prefix_lens) new_prefix_lens[b] = P;
     }
     return;
   }
-  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_keep, s_rows);
-  if (threadIdx.x == 0) {
+  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_keep, s_rows, slice);
+  if (threadIdx.x == 0 && slice == 0) {
     if (status) status[b] = DDT_REQ_OK;
     if (new_prefix_lens) new_prefix_lens[b] = P + alen;
   }
@@ -246,26 +280,33 @@ __global__ void __launch_bounds__(kCompactThreads) kv_compact_kernel(
 // ---------------------------------------------------------------------------
 // Accept fused with compaction.  [Race Conditions] "The Broader Significance"
 // defers fusing the compaction gather to a later phase, keeping it a separate
-// step.  Here one CTA per request walks the tree (thread 0,
-// the same walk as tree_accept_kernel) and then moves the accepted rows (all
-// threads, the same staging as kv_compact_kernel), so the path never leaves the
-// chip and one launch replaces two.  The walk always yields 1 <= alen <= q_len
-// and path entries in [0, q_len), so compaction can only fail on the prefix.
+// step.  Here the kCompactSlices CTAs of a request (one cluster) each walk the
+// tree (thread 0, the same walk as tree_accept_kernel) and then move their
+// slice of the accepted rows (the same staging as kv_compact_kernel), so the
+// path never leaves the chip and one launch replaces two; the first slice
+// publishes the walk's outputs.  The walk always yields 1 <= alen <= q_len and
+// path entries in [0, q_len), so compaction can only fail on the prefix.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kCompactThreads) accept_compact_kernel(
-    const int32_t* __restrict__ node_tokens, const int32_t* __restrict__ target_tokens,
-    const int32_t* __restrict__ next_token, const int32_t* __restrict__ next_sibling, int q_len,
-    uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope, int64_t ckv_bs, int64_t ckv_rs,
-    int64_t kr_bs, int64_t kr_rs, int capacity, const int32_t* prefix_lens,
-    int32_t* __restrict__ path, int32_t* __restrict__ accept_len, int32_t* __restrict__ bonus_token,
-    int32_t* __restrict__ accept_status, int32_t* new_prefix_lens,
-    int32_t* __restrict__ compact_status) {
-  extern __shared__ uint4 s_rows[];  // [alen][kRowVec]
+__global__ void __cluster_dims__(kCompactSlices, 1, 1) __launch_bounds__(kCompactThreads)
+    accept_compact_kernel(const int32_t* __restrict__ node_tokens,
+                          const int32_t* __restrict__ target_tokens,
+                          const int32_t* __restrict__ next_token,
+                          const int32_t* __restrict__ next_sibling, int q_len,
+                          uint16_t* __restrict__ c_kv, uint16_t* __restrict__ k_rope,
+                          int64_t ckv_bs, int64_t ckv_rs, int64_t kr_bs, int64_t kr_rs,
+                          int capacity, const int32_t* prefix_lens, int32_t* __restrict__ path,
+                          int32_t* __restrict__ accept_len, int32_t* __restrict__ bonus_token,
+                          int32_t* __restrict__ accept_status, int32_t* new_prefix_lens,
+                          int32_t* __restrict__ compact_status) {
+  extern __shared__ uint4 s_rows[];  // [alen][kSliceVec]
   __shared__ int32_t s_tok[DDT_MAX_Q_LEN], s_tgt[DDT_MAX_Q_LEN], s_first[DDT_MAX_Q_LEN],
       s_sib[DDT_MAX_Q_LEN], s_path[DDT_MAX_Q_LEN];
   __shared__ int s_alen, s_state;
-  const int b = blockIdx.x;
-  const int P = prefix_lens[b];  // read by every thread before the first barrier
+  const int b = blockIdx.x / kCompactSlices;
+  const int slice = blockIdx.x % kCompactSlices;
+  // Read by every thread of every slice before the cluster barrier below, so
+  // new_prefix_lens may be prefix_lens itself.
+  const int P = prefix_lens[b];
   const int64_t base = static_cast<int64_t>(b) * q_len;
   for (int k = threadIdx.x; k < q_len; k += kCompactThreads) {
     s_tok[k] = node_tokens[base + k];
@@ -278,25 +319,31 @@ __global__ void __launch_bounds__(kCompactThreads) accept_compact_kernel(
   if (threadIdx.x == 0) {
     int alen, cur;
     const int st = accept_walk(s_tok, s_tgt, s_first, s_sib, q_len, s_path, alen, cur);
-    accept_len[b] = alen;
-    if (bonus_token) bonus_token[b] = s_tgt[cur];
-    if (accept_status) accept_status[b] = st;
+    if (slice == 0) {
+      accept_len[b] = alen;
+      if (bonus_token) bonus_token[b] = s_tgt[cur];
+      if (accept_status) accept_status[b] = st;
+    }
     s_alen = alen;
     s_state = (P < 0 || static_cast<int64_t>(P) + q_len > capacity) ? DDT_REQ_BAD_PREFIX
                                                                      : DDT_REQ_OK;
   }
   __syncthreads();
   const int alen = s_alen;
-  for (int k = threadIdx.x; k < q_len; k += kCompactThreads) path[base + k] = s_path[k];
-  if (s_state != DDT_REQ_OK) {
-    if (threadIdx.x == 0) {
-      if (compact_status) compact_status[b] = s_state;
+  if (slice == 0)
+    for (int k = threadIdx.x; k < q_len; k += kCompactThreads) path[base + k] = s_path[k];
+  const int st = s_state;
+  // Every slice has read P and its tree arrays.
+  compact_cluster_sync();
+  if (st != DDT_REQ_OK) {
+    if (threadIdx.x == 0 && slice == 0) {
+      if (compact_status) compact_status[b] = st;
       if (new_prefix_lens) new_prefix_lens[b] = P;
     }
     return;
   }
-  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_path, s_rows);
-  if (threadIdx.x == 0) {
+  compact_rows(c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, b, P, alen, s_path, s_rows, slice);
+  if (threadIdx.x == 0 && slice == 0) {
     if (compact_status) compact_status[b] = DDT_REQ_OK;
     if (new_prefix_lens) new_prefix_lens[b] = P + alen;
   }
@@ -367,11 +414,11 @@ cudaError_t launch_kv_compact(uint16_t* c_kv, uint16_t* k_rope, int64_t ckv_bs, 
                               const int32_t* prefix_lens, const int32_t* path,
                               const int32_t* accept_len, int B, int q_len,
                               int32_t* new_prefix_lens, int32_t* status, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(q_len) * kRowVec * sizeof(uint4);
+  const size_t smem = static_cast<size_t>(q_len) * kSliceVec * sizeof(uint4);
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kv_compact_kernel),
-                                    static_cast<int>(DDT_MAX_Q_LEN * kRowVec * sizeof(uint4)), 0);
+                                    static_cast<int>(DDT_MAX_Q_LEN * kSliceVec * sizeof(uint4)), 0);
   if (e != cudaSuccess) return e;
-  kv_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
+  kv_compact_kernel<<<B * kCompactSlices, kCompactThreads, smem, stream>>>(
       c_kv, k_rope, ckv_bs, ckv_rs, kr_bs, kr_rs, capacity, prefix_lens, path, accept_len, q_len,
       new_prefix_lens, status);
   return cudaGetLastError();
@@ -384,11 +431,11 @@ cudaError_t launch_accept_compact(const int32_t* node_tokens, const int32_t* tar
                                   const int32_t* prefix_lens, int32_t* path, int32_t* accept_len,
                                   int32_t* bonus, int32_t* accept_status, int32_t* new_prefix_lens,
                                   int32_t* compact_status, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(q_len) * kRowVec * sizeof(uint4);
+  const size_t smem = static_cast<size_t>(q_len) * kSliceVec * sizeof(uint4);
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(accept_compact_kernel),
-                                    static_cast<int>(DDT_MAX_Q_LEN * kRowVec * sizeof(uint4)), 4);
+                                    static_cast<int>(DDT_MAX_Q_LEN * kSliceVec * sizeof(uint4)), 4);
   if (e != cudaSuccess) return e;
-  accept_compact_kernel<<<B, kCompactThreads, smem, stream>>>(
+  accept_compact_kernel<<<B * kCompactSlices, kCompactThreads, smem, stream>>>(
       node_tokens, target_tokens, next_token, next_sibling, q_len, c_kv, k_rope, ckv_bs, ckv_rs,
       kr_bs, kr_rs, capacity, prefix_lens, path, accept_len, bonus, accept_status,
       new_prefix_lens, compact_status);

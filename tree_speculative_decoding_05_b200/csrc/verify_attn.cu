@@ -35,10 +35,11 @@
 //     128-key tiles are the default.
 //   * Warp roles: warps 0-3 softmax and epilogue (thread t owns TMEM lane t, i.e.
 //     half of one query row); warps 4 and 8 TMA producers of the K rings of
-//     even and odd tiles, warp 6 the producer of the V ring; warps 5 and 9
+//     even and odd tiles, warp 6 the producer of the V ring; warps 5 and 10
 //     issue S = Q K^T for even and odd tiles and warp 7 issues O += P V (the
-//     even CTA of the pair issues for both).  Three issuing threads keep the
-//     tensor core fed while each waits on barriers or commits stages.
+//     even CTA of the pair issues for both); warp 9 idles.  Three issuing
+//     threads keep the tensor core fed while each waits on barriers or commits
+//     stages, and they sit on three different SM sub-partitions.
 //   * Online softmax in registers with exp2; the row maximum of the two half
 //     rows is exchanged through shared memory; O is rescaled lazily, only when
 //     the running maximum grows by more than 2^8.
@@ -69,14 +70,24 @@ namespace ddt {
 namespace va {
 // S = Q K^T issuers: tile G goes to issuer G % kQKIss, each with its own K ring
 // and its own K producer warp.
-#ifndef DDT_VERIFY_QK_ISSUERS
-#define DDT_VERIFY_QK_ISSUERS 2
+constexpr int kQKIss = 2;
+// Warp roles.  Warp w runs on sub-partition w % 4, and each sub-partition runs
+// one softmax warp (warps 0-3: TMEM lane quarter w).  The three threads that
+// issue MMAs sit on three different sub-partitions, so no two of them share a
+// scheduler: with both S issuers on one sub-partition the kernel ran 3-10 %
+// slower.  DDT_VERIFY_WARP_MAP 11 (default): 4 K producer 0 (and Q), 5 S issuer
+// 0, 6 V producer, 7 P V issuer, 8 K producer 1, 9 idle, 10 S issuer 1.
+// DDT_VERIFY_WARP_MAP 10: the same without the idle warp (6 S issuer 1, 9 V
+// producer).
+#ifndef DDT_VERIFY_WARP_MAP
+#define DDT_VERIFY_WARP_MAP 11
 #endif
-constexpr int kQKIss = DDT_VERIFY_QK_ISSUERS;
-static_assert(kQKIss == 2 || kQKIss == 3, "two or three S issuers");
-// Warps 0-3 softmax; 4 K producer 0 (and Q), 5 S issuer 0, 6 V producer, 7 P V
-// issuer, 8 K producer 1, 9 S issuer 1, 10 K producer 2, 11 S issuer 2.
-constexpr int kThreads = 32 * (6 + 2 * kQKIss);
+static_assert(DDT_VERIFY_WARP_MAP == 10 || DDT_VERIFY_WARP_MAP == 11, "warp map 10 or 11");
+constexpr int kWarpKProd0 = 4, kWarpSIss0 = 5, kWarpPVIss = 7, kWarpKProd1 = 8;
+constexpr int kWarpVProd = DDT_VERIFY_WARP_MAP == 11 ? 6 : 9;
+constexpr int kWarpSIss1 = DDT_VERIFY_WARP_MAP == 11 ? 10 : 6;
+constexpr int kWarpTmem = kWarpSIss0;  // allocates and frees the tensor memory
+constexpr int kThreads = 32 * DDT_VERIFY_WARP_MAP;
 constexpr int kSoftmaxThreads = 128;
 constexpr int kStageBytes = 8192;                  // Q chunk, P chunk, output box: 64 x 128 B
 // KV tile: kTK cache rows per tile; each CTA of the pair stages kKH of them for
@@ -265,7 +276,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_ckv_k,
                        const __grid_constant__ CUtensorMap tm_ckv_v,
                        const __grid_constant__ CUtensorMap tm_krope,
-                       const __grid_constant__ CUtensorMap tm_out, const VerifyParams p) {
+                       const __grid_constant__ CUtensorMap tm_out,
+                       const __grid_constant__ CUtensorMap tm_f32, const VerifyParams p) {
   using namespace va;
   const uint32_t rank = cluster_ctarank();
   const int cluster = static_cast<int>(blockIdx.x >> 1);
@@ -317,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init_cluster();
   }
-  if (warp == 5) {
+  if (warp == kWarpTmem) {
     tmem_alloc<2>(smem_u32(tmem_ptr_smem), kTmemCols);
     tmem_relinquish<2>();
   }
@@ -363,11 +375,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
   };
   const bool leader = rank == 0;
 
-  // K producer g: warp 4, 8, 10; S issuer g: the next warp (5, 9, 11).
-  const int qk_g = warp == 4 || warp == 5 ? 0 : warp == 8 || warp == 9 ? 1
-                   : warp == 10 || warp == 11 ? 2 : -1;
-  const bool k_producer = qk_g >= 0 && (warp & 1) == 0;
-  const bool s_issuer = qk_g >= 0 && (warp & 1) == 1;
+  // K producer g and S issuer g share ring g.
+  const int qk_g = warp == kWarpKProd0 || warp == kWarpSIss0   ? 0
+                   : warp == kWarpKProd1 || warp == kWarpSIss1 ? 1
+                                                               : -1;
+  const bool k_producer = warp == kWarpKProd0 || warp == kWarpKProd1;
+  const bool s_issuer = warp == kWarpSIss0 || warp == kWarpSIss1;
   if (k_producer) {
     // ---------------------------------------------- TMA: Q and the K rings
     // Lane 0 issues; producer g loads the K stages of tiles G with G % kQKIss == g
@@ -419,7 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 6) {
+  } else if (warp == kWarpVProd) {
     // ------------------------------------------------------------ TMA: V ring
     if (lane == 0) {
       Ring r;
@@ -498,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_wait(bar(kBarQKDone + g), 0, abort_flag);
     }
     __syncwarp();
-  } else if (warp == 7) {
+  } else if (warp == kWarpPVIss) {
     // ------------------------------------------------------- MMA: O += P V
     if (leader && lane == 0) {
       Ring r;
@@ -544,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
       mbar_wait(bar(kBarPVDone), 0, abort_flag);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 4) {
     // -------------------------------------------------------- softmax warps
     const int t = threadIdx.x;         // TMEM lane
     const int m = t & 63;              // row within this CTA (head)
@@ -762,39 +775,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           named_barrier_sync(2, kSoftmaxThreads);
         }
         if (hf == 0 && p.lse) p.lse[static_cast<int64_t>(row0) + m] = lse_nat;
-      } else {
-        if (node_valid) {
-          const int64_t row = (static_cast<int64_t>(b) * Q + node) * 64 + m;
-          const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+      } else if (node_valid) {
+        // fp32 output, or a split's normalised partial: also staged in shared
+        // memory and written with TMA tile stores (32 columns x 64 rows of fp32
+        // per box, 128-byte swizzle), in four rounds of 64 rows x 128 columns.
+        // Round r takes, from each thread's half row, the 64 columns
+        // 256 (r / 2) + 128 hf + 64 (r % 2) + [0, 64).
+        const int64_t rows_total = static_cast<int64_t>(p.B) * Q * 64;
+        const int64_t row0 = (static_cast<int64_t>(b) * Q + node) * 64;
+        const int grow0 = static_cast<int>(
+            p.write_partials ? (split + p.split_base) * rows_total + row0 : row0);
+        uint8_t* stage = base + kOffP;
+        const uint32_t stage_addr = base_addr + kOffP;
 #pragma unroll 1
-          for (int nh = 0; nh < 2; ++nh) {
+        for (int r = 0; r < 4; ++r) {
+          const int nh = r >> 1;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * q, o);
-              tmem_wait_ld();
-              const int col = 256 * nh + 128 * hf + 32 * q;
-              float4* dst =
-                  p.write_partials
-                      ? reinterpret_cast<float4*>(
-                            p.part_o +
-                            (static_cast<int64_t>(split + p.split_base) * rows_total + row) * 512 +
-                            col)
-                      : reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * 512 + col);
+          for (int qq = 0; qq < 2; ++qq) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + kTmemO + 128u * nh + 32u * (2 * (r & 1) + qq), o);
+            tmem_wait_ld();
+            // box 2 hf + qq, row m: 8 units of 16 bytes, 128-byte swizzle by row
+            uint8_t* rowp = stage + (2 * hf + qq) * kStageBytes + m * 128;
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                     __uint_as_float(o[4 * v + 2]) * inv,
-                                     __uint_as_float(o[4 * v + 3]) * inv);
+            for (int v = 0; v < 8; ++v) {
+              const float4 val = make_float4(__uint_as_float(o[4 * v]) * inv,
+                                             __uint_as_float(o[4 * v + 1]) * inv,
+                                             __uint_as_float(o[4 * v + 2]) * inv,
+                                             __uint_as_float(o[4 * v + 3]) * inv);
+              *reinterpret_cast<float4*>(rowp + ((v ^ (m & 7)) << 4)) = val;
             }
           }
-          if (hf == 0) {
-            if (p.write_partials)
-              p.part_lse[static_cast<int64_t>(split + p.split_base) * rows_total + row] = lse_nat;
-            else if (p.lse) p.lse[row] = lse_nat;
+          if (r == 3) tc_fence_before_sync();  // every read of O is done
+          fence_proxy_async_smem();
+          named_barrier_sync(2, kSoftmaxThreads);
+          // O has been read: the next item's first P V may overwrite it.
+          if (r == 3 && t == 0) mbar_arrive_cluster(o_free_leader);
+          if (t == 0) {
+            for (int k = 0; k < 4; ++k)
+              tma_store_3d(&tm_f32, stage_addr + k * kStageBytes,
+                           256 * nh + 128 * (k >> 1) + 64 * (r & 1) + 32 * (k & 1), grow0, 0);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging buffer may be written again
           }
+          named_barrier_sync(2, kSoftmaxThreads);
         }
-        // O has been read: the next item's first P V may overwrite it.
+        if (hf == 0) {
+          if (p.write_partials)
+            p.part_lse[static_cast<int64_t>(split + p.split_base) * rows_total + row0 + m] = lse_nat;
+          else if (p.lse) p.lse[row0 + m] = lse_nat;
+        }
+      } else {
+        // A node past q_len (odd q_len): nothing to write; release O.
         tc_fence_before_sync();
         named_barrier_sync(2, kSoftmaxThreads);
         if (t == 0) mbar_arrive_cluster(o_free_leader);
@@ -802,13 +834,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
     }
     if (t == 0) bulk_wait_group0();  // this CTA's output stores have completed
   }
+  // (an idle warp of the 11-warp map goes straight to the final barrier)
 
   // All MMAs of the pair are complete here (the softmax warps waited for the
   // last O commit, the issuer for its final commit); release tensor memory.
   __syncwarp();
   tc_fence_before_sync();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == kWarpTmem) {
     tc_fence_after_sync();
     tmem_dealloc<2>(tmem, kTmemCols);
   }
@@ -905,15 +938,16 @@ EncodeTiledFn encode_fn() {
 // 3-D bf16 map: dims {d0 (contiguous), d1, d2}, byte strides of d1 and d2, box
 // {64, box1, 1}, 128-byte swizzle, zero fill out of bounds.
 bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1) {
+              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t box0 = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  const cuuint32_t box[3] = {64, box1, 1};
+  const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return fn(m, dtype, 3, const_cast<void*>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -925,7 +959,7 @@ namespace {
 ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int write_partials,
                        int split_base, float* part_o, float* part_lse, cudaStream_t stream) {
   using namespace va;
-  CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out;
+  CUtensorMap m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out, m_f32;
   const uint64_t rows_q = static_cast<uint64_t>(a.q_len) * 64;
   const uint64_t B = static_cast<uint64_t>(a.B);
   const uint64_t cap = static_cast<uint64_t>(a.capacity);
@@ -940,6 +974,19 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
     ok = ok && make_map(&m_out, a.out, 512, out_rows, 1, 512 * 2, out_rows * 512 * 2, 64);
   else
     m_out = m_qlat;  // not read
+  // fp32 rows [.., 512] stored in 32 x 64 boxes: the output, or every partial of
+  // the workspace up to this pass's last split.
+  const uint64_t rows_total = static_cast<uint64_t>(a.B) * a.q_len * 64;
+  if (write_partials) {
+    const uint64_t prow = static_cast<uint64_t>(split_base + num_splits) * rows_total;
+    ok = ok && make_map(&m_f32, part_o, 512, prow, 1, 512 * 4, prow * 512 * 4, 64,
+                        CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32);
+  } else if (a.out_dtype == DDT_F32) {
+    ok = ok && make_map(&m_f32, a.out, 512, rows_total, 1, 512 * 4, rows_total * 512 * 4, 64,
+                        CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32);
+  } else {
+    m_f32 = m_qlat;  // not read
+  }
   if (!ok) return DDT_ERR_INVALID_ARG;
   if (ensure_smem_limit(reinterpret_cast<const void*>(verify_attn_kernel), kSmemBytes, 1) !=
       cudaSuccess)
@@ -968,7 +1015,7 @@ ddt_status launch_pass(const ddt_attn_args& a, int kv_mode, int num_splits, int 
   const int64_t slots = device_sm_count() / 2 > 0 ? device_sm_count() / 2 : 1;
   const int64_t grid = 2 * (items < slots ? items : slots);
   verify_attn_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
-      m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out, p);
+      m_qlat, m_qrope, m_ckv_k, m_ckv_v, m_krope, m_out, m_f32, p);
   return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
