@@ -872,26 +872,54 @@ __global__ void __launch_bounds__(256) verify_merge_kernel(const float* __restri
     split_range(T, n_cache, s, t0, t1);
     return t0 < t1;
   };
+  // The splits' lse values lane-parallel (split s on lane s % 32), their maximum
+  // and weights by warp shuffles; then the partial rows four splits at a time,
+  // every load of a group issued before its accumulation.  Absent splits (never
+  // written) and empty ones (lse = -inf) get weight 0 and are not read.
   float lmax = -INFINITY;
-  for (int s = 0; s < num_splits; ++s)
+  for (int s = lane; s < num_splits; s += 32)
     if (present(s)) lmax = fmaxf(lmax, part_lse[s * rows_total + row]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
   float acc[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) acc[k] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < num_splits; ++s) {
-    if (!present(s)) continue;
-    const float ls = part_lse[s * rows_total + row];
-    const float w = (ls == -INFINITY) ? 0.f : fast_exp2((ls - lmax) * va::kLog2e);
-    wsum += w;
-    const float4* src = reinterpret_cast<const float4*>(part_o + (s * rows_total + row) * 512);
+  for (int s0 = 0; s0 < num_splits; s0 += 32) {
+    const int s = s0 + lane;
+    float wl = 0.f;
+    if (s < num_splits && present(s)) {
+      const float ls = part_lse[s * rows_total + row];
+      wl = (ls == -INFINITY) ? 0.f : fast_exp2((ls - lmax) * va::kLog2e);
+    }
+    float wsum_c = wl;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 v = src[lane + 32 * k];
-      acc[4 * k] += w * v.x;
-      acc[4 * k + 1] += w * v.y;
-      acc[4 * k + 2] += w * v.z;
-      acc[4 * k + 3] += w * v.w;
+    for (int off = 16; off > 0; off >>= 1) wsum_c += __shfl_xor_sync(0xffffffffu, wsum_c, off);
+    wsum += wsum_c;
+    const int n = num_splits - s0 < 32 ? num_splits - s0 : 32;
+    for (int u0 = 0; u0 < n; u0 += 4) {
+      float w[4];
+      float4 v[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wu = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
+        w[u] = u0 + u < n ? wu : 0.f;
+        const float4* src = reinterpret_cast<const float4*>(
+            part_o + (static_cast<int64_t>(s0 + u0 + u) * rows_total + row) * 512);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          v[u][k] = w[u] != 0.f ? src[lane + 32 * k] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc[4 * k] += w[u] * v[u][k].x;
+          acc[4 * k + 1] += w[u] * v[u][k].y;
+          acc[4 * k + 2] += w[u] * v[u][k].z;
+          acc[4 * k + 3] += w[u] * v[u][k].w;
+        }
+      }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
