@@ -149,6 +149,24 @@ def test_kv_compact_at_scale():
     assert (ref[3] == 0).all()
 
 
+def test_kv_compact_in_place_prefix_update():
+    """new_prefix_lens = prefix_lens (the decode loop's in-place update): the
+    slices of a request must all read the old prefix before it is overwritten.
+    Every request of a 300-request batch moves rows; results bit for bit."""
+    B, Q = 300, 65
+    P = [int(x) for x in np.random.RandomState(5).randint(0, 400, size=B)]
+    c_kv, k_rope, Pv, path, alen, cap = _compact_case(B, Q, P, 17, "any")
+    ref = oracle.kv_compact(c_kv, k_rope, Pv, path, alen, capacity=cap)
+    ckv_t = torch.from_numpy(c_kv.view(np.int16)).cuda().view(torch.bfloat16)
+    kr_t = torch.from_numpy(k_rope.view(np.int16)).cuda().view(torch.bfloat16)
+    prefix = i32(Pv)
+    newp, status = ddt.kv_compact(ckv_t, kr_t, prefix, i32(path), i32(alen), new_prefix_lens=prefix)
+    assert newp.data_ptr() == prefix.data_ptr()
+    assert np.array_equal(ckv_t.view(torch.int16).cpu().numpy().view(np.uint16), ref[0])
+    assert np.array_equal(kr_t.view(torch.int16).cpu().numpy().view(np.uint16), ref[1])
+    assert np.array_equal(prefix.cpu().numpy(), ref[2]) and np.array_equal(status.cpu().numpy(), ref[3])
+
+
 def test_kv_compact_race_pattern_and_errors():
     """keep = [0, 2, 3] (the racing pattern) plus malformed requests."""
     B, Q = 4, 8
