@@ -269,6 +269,19 @@ def test_verify_attn_configs(cfg):
     compare_whole(out, lse, w, oracle, what=f"config {cfg} (whole output)")
 
 
+def test_verify_attn_whole_output_two_mask_words():
+    """q_len 128 (two mask words per node, 64 node pairs) with ragged prefixes and
+    an fp32 lse: every output row against the oracle."""
+    P = inputs.ragged_prefixes(4242, 4, 0, 3000)
+    w = inputs.make_workload("q128", 4242, 4, 128, P, want_lse=True,
+                             row_scale_range=(0.5, 2.0))
+    dw = DeviceWorkload(w)
+    out, lse, status = dw.verify()
+    torch.cuda.synchronize()
+    assert (status.cpu().numpy() == 0).all()
+    compare_whole(out, lse, w, oracle, what="4 x q128 ragged (whole output)")
+
+
 def test_step_configs_accept_and_compact():
     """Config 2 and 4 continue with tree_accept and kv_compact: bit-exact."""
     for cfg in (2, 4):

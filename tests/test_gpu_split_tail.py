@@ -83,3 +83,14 @@ def test_split_tail_requires_workspace():
     lib = ddt.load()
     assert lib.ddt_verify_attn_split_tail_workspace_size(a) > 0
     assert lib.ddt_verify_attn_split_tail(a, None) == ddt.DDT_ERR_INVALID_ARG
+
+
+def test_split_tail_whole_output_of_the_eight_request_workload():
+    """The prefix / tail split over every output row of the 8 x q_len 33 x prefix
+    1024 workload (16 896 rows), rel-L2 over the whole tensor."""
+    from gpu_helpers import compare_whole
+
+    w = inputs.config(1)
+    dw = DeviceWorkload(w)
+    out, lse = _split_tail(dw)
+    compare_whole(out, lse, w, oracle, what="split tail, config 1 (whole output)")
