@@ -241,31 +241,21 @@ __global__ void __launch_bounds__(kCompactThreads)
                       int32_t* __restrict__ status) {
   extern __shared__ uint4 s_rows[];  // [alen][kSliceVec]
   __shared__ int32_t s_keep[DDT_MAX_Q_LEN];
-  __shared__ int s_state;  // 0 ok, else status code
+  static_assert(DDT_MAX_Q_LEN <= kCompactThreads, "one thread per path entry");
   const int b = blockIdx.x / kCompactSlices;
   const int slice = blockIdx.x % kCompactSlices;
-  // In place: read by every thread of every slice before the cluster barrier
-  // below, so new_prefix_lens may be prefix_lens itself.
+  const int t = threadIdx.x;
+  // The prefix length, the accepted length and the whole path row are loaded
+  // together (one memory latency before the row copies can be addressed).
   const int P = prefix_lens[b];
   const int alen = accept_len[b];
-  if (threadIdx.x == 0) {
-    int st = DDT_REQ_OK;
-    if (alen < 1 || alen > q_len) st = DDT_REQ_BAD_LENGTH;
-    else if (P < 0 || static_cast<int64_t>(P) + q_len > capacity) st = DDT_REQ_BAD_PREFIX;
-    s_state = st;
-  }
-  __syncthreads();
-  if (s_state == DDT_REQ_OK) {
-    int bad = 0;
-    for (int i = threadIdx.x; i < alen; i += kCompactThreads) {
-      const int k = path[static_cast<int64_t>(b) * q_len + i];
-      s_keep[i] = k;
-      bad |= (k < 0 || k >= q_len);
-    }
-    if (__syncthreads_or(bad) && threadIdx.x == 0) s_state = DDT_REQ_BAD_INDEX;
-    __syncthreads();
-  }
-  const int st = s_state;
+  const int k = (t < q_len) ? path[static_cast<int64_t>(b) * q_len + t] : 0;
+  int st = DDT_REQ_OK;
+  if (alen < 1 || alen > q_len) st = DDT_REQ_BAD_LENGTH;
+  else if (P < 0 || static_cast<int64_t>(P) + q_len > capacity) st = DDT_REQ_BAD_PREFIX;
+  if (t < q_len) s_keep[t] = k;
+  const int bad = (st == DDT_REQ_OK) && t < alen && (k < 0 || k >= q_len);
+  if (__syncthreads_or(bad) && st == DDT_REQ_OK) st = DDT_REQ_BAD_INDEX;
   // Every slice has read P (and the same path, so the same verdict).
   if constexpr (kInPlace) compact_cluster_sync();
   if (st != DDT_REQ_OK) {
