@@ -15,7 +15,7 @@ namespace ddt {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSlots = 8;
+constexpr int kMaxSlots = 16;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

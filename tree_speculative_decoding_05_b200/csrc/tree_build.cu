@@ -31,10 +31,14 @@
 // pick is a lane-local maximum over the lane's key registers (fully unrolled,
 // so the keys never leave registers) and two warp-wide hardware reductions:
 // the maximum key, then the smallest slot holding it — no heap, no shuffle tree
-// and no memory access before the winner is known.  The log-probs and tokens a
+// and no memory access before the winner is known.  The kernel is instantiated
+// per number of key registers and launched with the fewest that hold a build's
+// 2 q_len - 1 slots, so the lane-local maximum and the key updates touch no
+// register that can only hold zero (at q_len 33: 3 instead of 8).  Every
+// log-prob is checked for finiteness first, and the log-probs and tokens a
 // build can touch (depth rows < min(D, q_len-1), ranks < min(K, q_len)) are
-// staged in shared memory first, in the same pass that checks every log-prob
-// for finiteness, so no pick waits on global memory.  The weights use
+// staged in shared memory with 32-bit index arithmetic, so no pick waits on
+// global memory.  The weights use
 // explicitly rounded float32 adds and subtracts (__fadd_rn / __fsub_rn), which
 // the compiler may neither contract nor reorder, so the result is bit-identical
 // to any float32 evaluation of the same expressions.  Each new node is linked
@@ -55,9 +59,11 @@ namespace ddt {
 namespace tb {
 // Dynamic shared memory bound: rows < q_len-1, ranks < q_len, float + int each.
 constexpr int kMaxStageBytes = (DDT_MAX_Q_LEN - 1) * DDT_MAX_Q_LEN * 8;
-// Candidate slots: at most 1 + 2 (q_len - 1) insertions; key registers per lane.
+// Candidate slots: at most 1 + 2 (q_len - 1) insertions; key registers per lane
+// (the kernel is instantiated for 1 .. kMaxKeyRegs registers and launched with
+// the fewest that hold 2 q_len - 1 slots).
 constexpr int kMaxSlots = 2 * DDT_MAX_Q_LEN;
-constexpr int kKeyRegs = kMaxSlots / 32;
+constexpr int kMaxKeyRegs = kMaxSlots / 32;
 static_assert(kMaxSlots % 32 == 0, "whole key registers");
 }  // namespace tb
 
@@ -71,12 +77,14 @@ __device__ __forceinline__ uint32_t weight_key(float w) {
 
 // Sets key register `reg` of a lane's candidate keys (reg is warp-uniform; the
 // unrolled compare keeps every index a constant, so the array stays in registers).
-__device__ __forceinline__ void set_key(uint32_t (&ck)[tb::kKeyRegs], int reg, uint32_t key) {
+template <int KR>
+__device__ __forceinline__ void set_key(uint32_t (&ck)[KR], int reg, uint32_t key) {
 #pragma unroll
-  for (int j = 0; j < tb::kKeyRegs; ++j)
+  for (int j = 0; j < KR; ++j)
     if (j == reg) ck[j] = key;
 }
 
+template <int KR>
 __global__ void __launch_bounds__(32) tree_build_kernel(
     const float* __restrict__ lp, const int32_t* __restrict__ tok,
     const int32_t* __restrict__ root_token, int D, int K, int q_len, int Dp, int Kp,
@@ -94,8 +102,8 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   __shared__ int32_t s_first[DDT_MAX_Q_LEN];  // first child (-1: none)
   __shared__ int32_t s_next[DDT_MAX_Q_LEN];   // next sibling (-1: none)
   __shared__ int32_t s_last[DDT_MAX_Q_LEN];   // newest child so far (-1: none)
-  __shared__ float s_cw[tb::kMaxSlots];       // candidate weight per slot
-  __shared__ int32_t s_cm[tb::kMaxSlots];     // candidate depth | rank << 8 | parent << 16
+  // per candidate slot: its weight's bits, and depth | rank << 8 | parent << 16
+  __shared__ uint2 s_cand[tb::kMaxSlots];
 
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
@@ -103,19 +111,15 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   const float* L = lp + b * DK;
   const int32_t* T = tok + b * DK;
 
-  // One pass over the drafts: every log-prob must be finite (a NaN would make
-  // the arg-max order-dependent), and the entries a build can read are staged.
+  // Every log-prob must be finite (a NaN would make the arg-max order-dependent);
+  // then the entries a build can read are staged (Dp * Kp < 2^14: 32-bit indexes).
   bool bad = false;
 #pragma unroll 4
-  for (int64_t e = lane; e < DK; e += 32) {
-    const float v = L[e];
-    bad |= !isfinite(v);
-    const int64_t d = e / K;
-    const int64_t r = e - d * K;
-    if (d < Dp && r < Kp) {
-      s_lp[d * Kp + r] = v;
-      s_tok[d * Kp + r] = T[e];
-    }
+  for (int64_t e = lane; e < DK; e += 32) bad |= !isfinite(L[e]);
+  for (int e = lane; e < Dp * Kp; e += 32) {
+    const int d = e / Kp, r = e - d * Kp;
+    s_lp[e] = L[static_cast<int64_t>(d) * K + r];
+    s_tok[e] = T[static_cast<int64_t>(d) * K + r];
   }
   bad = __any_sync(0xffffffffu, bad);
   for (int i = lane; i < q_len; i += 32) {
@@ -133,9 +137,9 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
 
   // Candidate keys: slot s in lane s % 32, register s / 32 (0 = empty).  Every
   // register index below is a compile-time constant, so ck stays in registers.
-  uint32_t ck[tb::kKeyRegs];
+  uint32_t ck[KR];
 #pragma unroll
-  for (int j = 0; j < tb::kKeyRegs; ++j) ck[j] = 0u;
+  for (int j = 0; j < KR; ++j) ck[j] = 0u;
   int n_slots = 0;
   // Inserts one candidate: its key in the slot's lane, weight and metadata by lane 0.
 #define DDT_TB_INSERT(w_, meta_)                                   \
@@ -143,10 +147,8 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     const int sl_ = n_slots++;                                     \
     const float wv_ = (w_);                                        \
     if (lane == (sl_ & 31)) set_key(ck, sl_ >> 5, weight_key(wv_)); \
-    if (lane == 0) {                                               \
-      s_cw[sl_] = wv_;                                             \
-      s_cm[sl_] = (meta_);                                         \
-    }                                                              \
+    if (lane == 0)                                                 \
+      s_cand[sl_] = make_uint2(__float_as_uint(wv_), (meta_));     \
   } while (0)
   if (!bad && q_len > 1) DDT_TB_INSERT(__fadd_rn(0.0f, s_lp[0]), 1 | (0 << 8) | (0 << 16));
   __syncwarp();
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     uint32_t bk = 0u;
     uint32_t bs = 0xffffffffu;
 #pragma unroll
-    for (int j = 0; j < tb::kKeyRegs; ++j) {
+    for (int j = 0; j < KR; ++j) {
       if (ck[j] > bk) {
         bk = ck[j];
         bs = static_cast<uint32_t>(j * 32 + lane);
@@ -168,8 +170,9 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     if (kmax == 0u) break;  // no candidate left
     const uint32_t win = __reduce_min_sync(0xffffffffu, bk == kmax ? bs : 0xffffffffu);
     if (lane == static_cast<int>(win & 31u)) set_key(ck, static_cast<int>(win >> 5), 0u);
-    const float bw = s_cw[win];
-    const int meta = s_cm[win];
+    const uint2 cand = s_cand[win];
+    const float bw = __uint_as_float(cand.x);
+    const int meta = static_cast<int>(cand.y);
     const int d = meta & 0xff, r = (meta >> 8) & 0xff, par = meta >> 16;
     const int node = n++;
     if (lane == 0) {
@@ -253,12 +256,22 @@ cudaError_t launch_tree_build(const float* lp, const int32_t* tok, const int32_t
   const int Dp = D < q_len - 1 ? D : q_len - 1;
   const int Kp = K < q_len ? K : q_len;
   const size_t smem = tree_build_smem_bytes(D, K, q_len);
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(tree_build_kernel),
-                                    tb::kMaxStageBytes, 3);
+  // the fewest key registers per lane that hold the 2 q_len - 1 candidate slots
+  const int kr = (2 * q_len - 1 + 31) / 32;
+  using Kernel = void (*)(const float*, const int32_t*, const int32_t*, int, int, int, int, int,
+                          int32_t*, int32_t*, int32_t*, float*, int32_t*, int32_t*, uint64_t*,
+                          int32_t*, int32_t*);
+  static constexpr Kernel kKernels[tb::kMaxKeyRegs] = {
+      tree_build_kernel<1>, tree_build_kernel<2>, tree_build_kernel<3>, tree_build_kernel<4>,
+      tree_build_kernel<5>, tree_build_kernel<6>, tree_build_kernel<7>, tree_build_kernel<8>};
+  static_assert(tb::kMaxKeyRegs == 8, "one instantiation per key-register count");
+  if (kr < 1 || kr > tb::kMaxKeyRegs) return cudaErrorInvalidValue;
+  const Kernel k = kKernels[kr - 1];
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(k), tb::kMaxStageBytes, 8 + kr - 1);
   if (e != cudaSuccess) return e;
-  tree_build_kernel<<<B, 32, smem, stream>>>(lp, tok, root_token, D, K, q_len, Dp > 0 ? Dp : 0,
-                                             Kp, parents, node_tokens, depth, logw, next_token,
-                                             next_sibling, mask, n_nodes, status);
+  k<<<B, 32, smem, stream>>>(lp, tok, root_token, D, K, q_len, Dp > 0 ? Dp : 0, Kp, parents,
+                             node_tokens, depth, logw, next_token, next_sibling, mask, n_nodes,
+                             status);
   return cudaGetLastError();
 }
 
