@@ -90,6 +90,17 @@ def test_tree_build_extreme_sizes():
     _check(lp1, tok1, root1, 128)  # a single candidate, then 126 padding slots
 
 
+@pytest.mark.parametrize("Q", [16, 17, 32, 33, 48, 49, 64, 65, 80, 81, 96, 97, 112, 113, 127])
+def test_tree_build_every_key_register_count(Q):
+    """The kernel is instantiated per number of candidate-key registers (1 to 8 per
+    lane, the fewest holding 2 Q - 1 slots) and per nodes per lane; these budgets
+    sit on both sides of every switch.  With D and K above Q every pick but the
+    last inserts two candidates, so the slot count reaches its bound."""
+    lp, tok, root = _draft(3000 + Q, 4, 130, 130)
+    g = _check(lp, tok, root, Q)
+    assert (g["n_nodes"] == Q).all()
+
+
 def test_tree_build_non_finite_logprobs():
     lp, tok, root = _draft(82, 6, 15, 8)
     lp[1, 14, 7] = np.nan

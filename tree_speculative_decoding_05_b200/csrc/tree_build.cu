@@ -41,11 +41,13 @@
 // global memory.  The weights use
 // explicitly rounded float32 adds and subtracts (__fadd_rn / __fsub_rn), which
 // the compiler may neither contract nor reorder, so the result is bit-identical
-// to any float32 evaluation of the same expressions.  Each new node is linked
-// as the newest child of its parent as it is created, which gives the retrieve
-// pointers (first child, next sibling) without a search.  After the expansion
-// the lanes build, one node each, the visibility words and the padding, and
-// write everything coalesced.
+// to any float32 evaluation of the same expressions.  A pick's only store is
+// the new node's record (weight, depth, rank, parent), by lane 0.  After the
+// expansion the lanes derive the retrieve pointers from the parents in one
+// pass (a node's first child is the earliest node it parents, its next sibling
+// the earliest later node with the same parent), then build, one node each,
+// the tokens, the visibility words and the padding, and write everything
+// coalesced.
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -95,13 +97,8 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   extern __shared__ __align__(16) unsigned char tb_smem[];
   float* s_lp = reinterpret_cast<float*>(tb_smem);                   // [Dp][Kp]
   int32_t* s_tok = reinterpret_cast<int32_t*>(tb_smem) + Dp * Kp;   // [Dp][Kp]
-  __shared__ int32_t s_par[DDT_MAX_Q_LEN];
-  __shared__ int32_t s_ntok[DDT_MAX_Q_LEN];
-  __shared__ int32_t s_dep[DDT_MAX_Q_LEN];
-  __shared__ float s_lw[DDT_MAX_Q_LEN];
-  __shared__ int32_t s_first[DDT_MAX_Q_LEN];  // first child (-1: none)
-  __shared__ int32_t s_next[DDT_MAX_Q_LEN];   // next sibling (-1: none)
-  __shared__ int32_t s_last[DDT_MAX_Q_LEN];   // newest child so far (-1: none)
+  // per node: its weight's bits, and depth | rank << 8 | parent << 16 (root: parent -1)
+  __shared__ uint2 s_node[DDT_MAX_Q_LEN];
   // per candidate slot: its weight's bits, and depth | rank << 8 | parent << 16
   __shared__ uint2 s_cand[tb::kMaxSlots];
 
@@ -122,17 +119,7 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     s_tok[e] = T[static_cast<int64_t>(d) * K + r];
   }
   bad = __any_sync(0xffffffffu, bad);
-  for (int i = lane; i < q_len; i += 32) {
-    s_first[i] = -1;
-    s_next[i] = -1;
-    s_last[i] = -1;
-  }
-  if (lane == 0) {
-    s_par[0] = -1;
-    s_ntok[0] = root_token[b];
-    s_dep[0] = 0;
-    s_lw[0] = 0.0f;
-  }
+  if (lane == 0) s_node[0] = make_uint2(0u, 0xffff0000u);  // weight +0, depth 0, parent -1
   __syncwarp();
 
   // Candidate keys: slot s in lane s % 32, register s / 32 (0 = empty).  Every
@@ -175,17 +162,7 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
     const int meta = static_cast<int>(cand.y);
     const int d = meta & 0xff, r = (meta >> 8) & 0xff, par = meta >> 16;
     const int node = n++;
-    if (lane == 0) {
-      s_par[node] = par;
-      s_ntok[node] = s_tok[(d - 1) * Kp + r];
-      s_dep[node] = d;
-      s_lw[node] = bw;
-      // node is the newest child of par: the first one, or the next sibling of the last
-      const int prev = s_last[par];
-      if (prev < 0) s_first[par] = node;
-      else s_next[prev] = node;
-      s_last[par] = node;
-    }
+    if (lane == 0) s_node[node] = cand;
     if (n == q_len) break;  // budget reached: nothing more will be picked
     if (d < D) DDT_TB_INSERT(__fadd_rn(bw, s_lp[d * Kp]), (d + 1) | (0 << 8) | (node << 16));
     if (r + 1 < K) {
@@ -197,21 +174,50 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
 #undef DDT_TB_INSERT
   __syncwarp();
 
+  // Retrieve pointers: node i's first child is the earliest node whose parent is
+  // i, its next sibling the earliest later node with i's parent (nodes are
+  // numbered in creation order).  Lane l holds nodes l, l + 32, ...; one
+  // broadcast read of each node's parent serves every lane.
+  constexpr int kNodesPerLane = (KR + 1) / 2;  // q_len <= 16 KR
+  int my_par[kNodesPerLane], my_first[kNodesPerLane], my_sib[kNodesPerLane];
+#pragma unroll
+  for (int k = 0; k < kNodesPerLane; ++k) {
+    const int i = lane + 32 * k;
+    my_par[k] = i < n ? static_cast<int>(s_node[i].y) >> 16 : -2;
+    my_first[k] = -1;
+    my_sib[k] = -1;
+  }
+  for (int j = 1; j < n; ++j) {
+    const int pj = static_cast<int>(s_node[j].y) >> 16;
+#pragma unroll
+    for (int k = 0; k < kNodesPerLane; ++k) {
+      const int i = lane + 32 * k;
+      if (pj == i && my_first[k] < 0) my_first[k] = j;
+      if (j > i && pj == my_par[k] && my_sib[k] < 0) my_sib[k] = j;
+    }
+  }
+
   // Per node: padding, retrieve pointers, visibility words; coalesced writes.
   const int W = (q_len + 63) >> 6;
   const int64_t row0 = static_cast<int64_t>(b) * q_len;
-  for (int i = lane; i < q_len; i += 32) {
+#pragma unroll
+  for (int k = 0; k < kNodesPerLane; ++k) {
+    const int i = lane + 32 * k;
+    if (i >= q_len) break;
     int p, t, dd, first = -1, sib = -1;
     float w;
     uint64_t w0 = 0, w1 = 0;
     if (i < n) {
-      p = s_par[i];
-      t = s_ntok[i];
-      dd = s_dep[i];
-      w = s_lw[i];
-      first = s_first[i];
-      sib = s_next[i];  // -1 for the root, which is no one's child
-      for (int a = i, steps = 0; a >= 0 && steps <= i; a = s_par[a], ++steps) {
+      const uint2 rec = s_node[i];
+      const int meta = static_cast<int>(rec.y);
+      p = meta >> 16;
+      dd = meta & 0xff;
+      t = i == 0 ? root_token[b] : s_tok[(dd - 1) * Kp + ((meta >> 8) & 0xff)];
+      w = __uint_as_float(rec.x);
+      first = my_first[k];
+      sib = my_sib[k];  // -1 for the root, which is no one's child
+      for (int a = i, steps = 0; a >= 0 && steps <= i;
+           a = static_cast<int>(s_node[a].y) >> 16, ++steps) {
         if (a < 64) w0 |= 1ull << a;
         else w1 |= 1ull << (a - 64);
       }
