@@ -34,11 +34,11 @@
 // and no memory access before the winner is known.  The kernel is instantiated
 // per number of key registers and launched with the fewest that hold a build's
 // 2 q_len - 1 slots, so the lane-local maximum and the key updates touch no
-// register that can only hold zero (at q_len 33: 3 instead of 8).  Every
-// log-prob is checked for finiteness first, and the log-probs and tokens a
-// build can touch (depth rows < min(D, q_len-1), ranks < min(K, q_len)) are
-// staged in shared memory with 32-bit index arithmetic, so no pick waits on
-// global memory.  The weights use
+// register that can only hold zero (at q_len 33: 3 instead of 8).  The
+// log-probs and tokens a build can touch (depth rows < min(D, q_len-1), ranks <
+// min(K, q_len)) are staged in shared memory, loaded together and checked for
+// finiteness on the way, and the other log-probs are only checked, so no pick
+// waits on global memory.  The weights use
 // explicitly rounded float32 adds and subtracts (__fadd_rn / __fsub_rn), which
 // the compiler may neither contract nor reorder, so the result is bit-identical
 // to any float32 evaluation of the same expressions.  A pick's only store is
@@ -108,16 +108,30 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
   const float* L = lp + b * DK;
   const int32_t* T = tok + b * DK;
 
-  // Every log-prob must be finite (a NaN would make the arg-max order-dependent);
-  // then the entries a build can read are staged (Dp * Kp < 2^14: 32-bit indexes).
+  const int root = lane == 0 ? root_token[b] : 0;  // used after the expansion
+  // Every log-prob must be finite (a NaN would make the arg-max order-dependent).
+  // The entries a build can read (rows d < Dp, ranks r < Kp; Dp * Kp < 2^14, so
+  // 32-bit indexes) are staged, their log-probs and tokens loaded together; then
+  // the rest of each staged row (ranks Kp .. K-1) and the rows from Dp on are
+  // only checked.
   bool bad = false;
 #pragma unroll 4
-  for (int64_t e = lane; e < DK; e += 32) bad |= !isfinite(L[e]);
   for (int e = lane; e < Dp * Kp; e += 32) {
     const int d = e / Kp, r = e - d * Kp;
-    s_lp[e] = L[static_cast<int64_t>(d) * K + r];
+    const float v = L[static_cast<int64_t>(d) * K + r];
     s_tok[e] = T[static_cast<int64_t>(d) * K + r];
+    bad |= !isfinite(v);
+    s_lp[e] = v;
   }
+  if (K > Kp) {
+    const int Kr = K - Kp;
+    for (int64_t e = lane; e < static_cast<int64_t>(Dp) * Kr; e += 32) {
+      const int64_t d = e / Kr;
+      bad |= !isfinite(L[d * K + Kp + (e - d * Kr)]);
+    }
+  }
+#pragma unroll 4
+  for (int64_t e = static_cast<int64_t>(Dp) * K + lane; e < DK; e += 32) bad |= !isfinite(L[e]);
   bad = __any_sync(0xffffffffu, bad);
   if (lane == 0) s_node[0] = make_uint2(0u, 0xffff0000u);  // weight +0, depth 0, parent -1
   __syncwarp();
@@ -212,7 +226,7 @@ __global__ void __launch_bounds__(32) tree_build_kernel(
       const int meta = static_cast<int>(rec.y);
       p = meta >> 16;
       dd = meta & 0xff;
-      t = i == 0 ? root_token[b] : s_tok[(dd - 1) * Kp + ((meta >> 8) & 0xff)];
+      t = i == 0 ? root : s_tok[(dd - 1) * Kp + ((meta >> 8) & 0xff)];
       w = __uint_as_float(rec.x);
       first = my_first[k];
       sib = my_sib[k];  // -1 for the root, which is no one's child
