@@ -1,6 +1,7 @@
 // api.cu — the extern "C" entry points of libddt: host-side argument checks,
 // then one launch per call on the caller's stream.  No entry point allocates
 // device memory or synchronises the host.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -16,6 +17,8 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSlots = 16;
+constexpr int kMaxContexts = 64;
+static_assert(kMaxSlots <= 32, "one bit per slot");
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -45,20 +48,70 @@ int device_sm_count() {
   return n;
 }
 
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct DriverFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+const DriverFns& driver_fns() {
+  static DriverFns fns;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  return fns;
+}
+
+}  // namespace
+
+unsigned long long current_context_id() {
+  const DriverFns& f = driver_fns();
+  if (!f.get_current || !f.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// A function attribute belongs to the function as loaded in one context (a
+// context that is reset or replaced loads the module afresh), so what has been
+// set is remembered per context ID: one bit per slot.
 cudaError_t ensure_smem_limit(const void* func, int bytes, int slot) {
   static std::mutex mu;
-  static bool done[kMaxDevices][kMaxSlots] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices || slot < 0 || slot >= kMaxSlots)
+  static unsigned long long ctx_id[kMaxContexts] = {};
+  static uint32_t done[kMaxContexts] = {};
+  static int next = 0;
+  const unsigned long long id = current_context_id();
+  if (id == 0 || slot < 0 || slot >= kMaxSlots)  // nothing to key a cache on
     return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   std::lock_guard<std::mutex> lock(mu);
-  if (!done[dev][slot]) {
-    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    done[dev][slot] = true;
+  int i = 0;
+  while (i < kMaxContexts && ctx_id[i] != id) ++i;
+  if (i < kMaxContexts && ((done[i] >> slot) & 1u)) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (i == kMaxContexts) {  // a context not seen yet takes the oldest entry
+    i = next;
+    next = (next + 1) % kMaxContexts;
+    ctx_id[i] = id;
+    done[i] = 0;
   }
+  done[i] |= 1u << slot;
   return cudaSuccess;
 }
 

@@ -71,7 +71,12 @@ ddt_status launch_verify_attn_split_tail(const ddt_attn_args& a, int prefix_spli
 
 int device_sm_count();
 
-// Sets the dynamic shared-memory limit of `func` on the current device once.
+// Sets the dynamic shared-memory limit of `func` once per CUDA context (`slot`
+// names the function, 0 .. 15).
 cudaError_t ensure_smem_limit(const void* func, int bytes, int slot);
+
+// Unique ID of the calling thread's current CUDA context (0 if there is none or
+// the driver cannot say).  IDs are never reused within a process.
+unsigned long long current_context_id();
 
 }  // namespace ddt

@@ -39,50 +39,16 @@
 #include <mutex>
 
 #include "ddt.h"
+#include "ddt_internal.h"
 
 namespace {
+
+using ddt::current_context_id;
 
 constexpr size_t kScratchBytes = static_cast<size_t>(32) << 20;
 constexpr int kMaxContexts = 64;
 
 static __device__ __align__(256) unsigned char g_verify_scratch[kScratchBytes];
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-struct DriverFns {
-  CtxGetCurrentFn get_current = nullptr;
-  CtxGetIdFn get_id = nullptr;
-};
-
-const DriverFns& driver_fns() {
-  static DriverFns fns;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fns.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fns.get_id = reinterpret_cast<CtxGetIdFn>(p);
-  });
-  return fns;
-}
-
-// Unique ID of the calling thread's current context (0 if there is none or the
-// driver cannot say).  IDs are never reused within a process.
-unsigned long long current_context_id() {
-  const DriverFns& f = driver_fns();
-  if (!f.get_current || !f.get_id) return 0;
-  CUcontext ctx = nullptr;
-  if (f.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
-  unsigned long long id = 0;
-  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
-  return id;
-}
 
 std::mutex g_scratch_mu;
 unsigned long long g_ctx_id[kMaxContexts] = {};
