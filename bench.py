@@ -538,7 +538,9 @@ def per_config_report(configs, peaks, device, preloaded=None):
     in one CUDA graph and the replay is timed with CUDA events on the launching
     stream, median of 5 replays (n = 100, or 20 for calls over 0.5 ms).  When the
     workload's inputs are under twice the L2, a 256 MB read precedes every call
-    and a graph of the writes alone is timed and subtracted.  Reported: µs per
+    and a graph of the writes alone is timed and subtracted; those workloads'
+    calls are also timed with a warm L2 (no read between calls), reported beside
+    them as `calls_us_warm_l2`.  Reported: µs per
     call of build_mask, verify_attn (with its split merge), tree_accept and
     kv_compact; verify TFLOP/s as a fraction of the burst and the sustained bf16
     peak; the KV stream's and the compaction's GB/s."""
@@ -585,7 +587,7 @@ def per_config_report(configs, peaks, device, preloaded=None):
             "kv_compact": lambda: ddt.kv_compact(c_kv, k_rope, prefix, path, alen,
                                                  new_prefix_lens=newp),
         }
-        us = {}
+        us, us_warm = {}, {}
         for name, fn in calls.items():
             for _ in range(5):
                 fn()
@@ -595,6 +597,8 @@ def per_config_report(configs, peaks, device, preloaded=None):
             torch.cuda.synchronize()
             n = 20 if time.perf_counter() - t0 > 0.5e-3 else 100
             us[name] = graph_time_us(fn, n, fl, reps=5)
+            if fl is not None:
+                us_warm[name] = graph_time_us(fn, n, None, reps=5)
         torch.cuda.synchronize()
         path_h, alen_h = path.cpu().numpy(), alen.cpu().numpy()
         moved = sum(int((path_h[b, :alen_h[b]] != np.arange(alen_h[b])).sum()) for b in range(B))
@@ -604,6 +608,7 @@ def per_config_report(configs, peaks, device, preloaded=None):
             "workload": w.name, "B": B, "q_len": Q, "prefix_max": max_prefix,
             "out": w.out_dtype, "lse": bool(w.want_lse), "kv_splits": splits,
             "calls_us": us,
+            **({"calls_us_warm_l2": us_warm} if us_warm else {}),
             "verify_gflop": flops / 1e9,
             "verify_tflops": tflops,
             "verify_frac_burst": tflops / peak_b,
