@@ -177,18 +177,70 @@ def record_traffic(csv_path: str, command: str) -> int:
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons while running: nvidia-smi every
+    100 ms, and NVML in-process every ~2 ms.  A timed region of a few tens of ms
+    falls between nvidia-smi's samples, so the summary takes the NVML samples
+    inside the region marked by begin() / end() when there are at least three,
+    else the nvidia-smi samples."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits and the names nvidia-smi gives them
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                   0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, device=None):
         self.gpu = gpu_index
+        self.device = device
         self.proc = None
         self.lines: list[str] = []
+        self.nvml_samples: list[tuple[float, float, int]] = []  # (time, SM MHz, reasons)
+        self.nvml_max = None
+        self.region = (None, None)
+        self._stop = threading.Event()
+        self._nvml_thread = None
+
+    def _nvml_start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            if self.device is not None:
+                import torch
+                pr = torch.cuda.get_device_properties(self.device)
+                bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+                except pynvml.NVMLError:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu))
+            self.nvml_max = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            return
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    rs = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    self.nvml_samples.append((time.perf_counter(), mhz, rs))
+                except Exception:
+                    return
+                time.sleep(0.002)
+
+        self._nvml_thread = threading.Thread(target=poll, daemon=True)
+        self._nvml_thread.start()
+
+    def begin(self):
+        self.region = (time.perf_counter(), None)
+
+    def end(self):
+        self.region = (self.region[0], time.perf_counter())
 
     def __enter__(self):
+        self._nvml_start()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
@@ -220,8 +272,26 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        self._stop.set()
+        if self._nvml_thread is not None:
+            self._nvml_thread.join(timeout=1.0)
 
     def summary(self):
+        t0, t1 = self.region
+        inside = [(m, r) for (t, m, r) in self.nvml_samples
+                  if t0 is not None and t1 is not None and t0 <= t <= t1]
+        if len(inside) >= 3:
+            reasons = set()
+            for _, r in inside:
+                for bit, name in self.REASON_BITS.items():
+                    if r & bit:
+                        reasons.add(name)
+            return {"sm_mhz": statistics.median(m for m, _ in inside),
+                    "sm_max_mhz": self.nvml_max, "reasons": sorted(reasons),
+                    "samples": len(inside), "source": "NVML every ~2 ms inside the timed region"}
+        return self._smi_summary()
+
+    def _smi_summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
@@ -239,7 +309,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi every 100 ms around the timed region"}
 
 
 def physical_gpu_index(local: int) -> str:
@@ -966,14 +1036,16 @@ def main(argv=None) -> int:
         dist.barrier()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(physical_gpu_index(local)) as clocks:
+    with ClockSampler(physical_gpu_index(local), device) as clocks:
         torch.cuda.synchronize()
+        clocks.begin()
         t_start.record(stream)
         for k in range(args.steps):
             flush_l2(k)
             step(evs[k])
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.end()
     if world > 1:
         dist.barrier()
     if flush is None:
@@ -1132,7 +1204,8 @@ def main(argv=None) -> int:
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
-                       "reasons": clk["reasons"]},
+                       "reasons": clk["reasons"], "samples": clk.get("samples"),
+                       "source": clk.get("source")},
             "faults": faults,
             "statuses_ok": statuses_ok,
         }

@@ -58,3 +58,25 @@ def test_traffic_record_from_ncu_raw_csv(tmp_path, monkeypatch):
     rec["kernel_source_sha256"] = "0" * 64
     rec_path.write_text(json.dumps(rec))
     assert bench.measured_traffic(2) is None
+
+
+def test_clock_summary_takes_samples_inside_the_timed_region():
+    """The NVML samples inside the marked region decide the clock summary (median
+    SM MHz, the union of the throttle reasons); with fewer than three of them the
+    nvidia-smi samples do."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    c = bench.ClockSampler("0")
+    c.nvml_max = 1965.0
+    c.region = (10.0, 10.05)
+    c.nvml_samples = [(9.99, 1965.0, 0), (10.01, 1500.0, 0x4), (10.02, 1520.0, 0x4),
+                      (10.03, 1480.0, 0x4 | 0x40), (10.06, 1965.0, 0)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1500.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    c.region = (10.0, 10.015)
+    c.lines = ["0, 1965, 1965, 300, 0x0, Not Active, Not Active, Not Active, Active"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
+    assert s["source"].startswith("nvidia-smi")
