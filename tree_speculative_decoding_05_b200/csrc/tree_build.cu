@@ -38,10 +38,10 @@
 // log-probs and tokens a build can touch (depth rows < min(D, q_len-1), ranks <
 // min(K, q_len)) are staged in shared memory, loaded together and checked for
 // finiteness on the way, and the other log-probs are only checked, so no pick
-// waits on global memory.  The weights use
-// explicitly rounded float32 adds and subtracts (__fadd_rn / __fsub_rn), which
-// the compiler may neither contract nor reorder, so the result is bit-identical
-// to any float32 evaluation of the same expressions.  A pick's only store is
+// waits on global memory.  The weights use explicitly rounded float32 adds and
+// subtracts (__fadd_rn / __fsub_rn), which the compiler may neither contract
+// nor reorder, so the result is bit-identical to any float32 evaluation of the
+// same expressions.  A pick's only store is
 // the new node's record (weight, depth, rank, parent), by lane 0.  After the
 // expansion the lanes derive the retrieve pointers from the parents in one
 // pass (a node's first child is the earliest node it parents, its next sibling
