@@ -168,18 +168,23 @@ def test_kv_compact_in_place_prefix_update():
 
 
 def test_kv_compact_race_pattern_and_errors():
-    """keep = [0, 2, 3] (the racing pattern) plus malformed requests."""
-    B, Q = 4, 8
-    c_kv, k_rope, Pv, path, alen, cap = _compact_case(B, Q, [5, 5, 5, 5], 3, "identity")
+    """keep = [0, 2, 3] (the racing pattern) plus malformed requests: every error
+    status, and bad entries past the accepted length, which are never read."""
+    B, Q = 8, 8
+    c_kv, k_rope, Pv, path, alen, cap = _compact_case(B, Q, [5] * B, 3, "identity")
     path[0, :3] = [0, 2, 3]; alen[0] = 3
     alen[1] = 0                                  # bad length
     path[2, :2] = [0, 99]; alen[2] = 2            # bad index
     Pv[3] = cap                                  # prefix past capacity
+    alen[4] = Q + 1                              # bad length (too long)
+    Pv[5] = -1                                   # negative prefix
+    path[6, :3] = [0, 2, 1]; path[6, 3:] = [-7, 99, 1000, -1, 8]; alen[6] = 3  # junk after alen
+    path[7, :2] = [0, -1]; alen[7] = 2            # negative index
     ref = oracle.kv_compact(c_kv, k_rope, Pv, path, alen, capacity=cap)
     got = _run_compact(c_kv, k_rope, Pv, path, alen, cap)
     for g, r, name in zip(got, ref, ("c_kv", "k_rope", "new_prefix", "status")):
         assert np.array_equal(g, r), name
-    assert list(ref[3]) == [0, 5, 2, 4]
+    assert list(ref[3]) == [0, 5, 2, 4, 5, 4, 0, 2]
 
 
 # ---------------------------------------------------------------------------
