@@ -215,7 +215,8 @@ typedef struct ddt_attn_args {
   int64_t ckv_batch_stride, ckv_row_stride; /* elements                         */
   int64_t kr_batch_stride, kr_row_stride;   /* elements                         */
   const uint64_t* mask; /* uint64 [B, q_len, W] from ddt_build_mask              */
-  float softmax_scale;
+  float softmax_scale; /* > 0 and finite (e.g. 1/sqrt(576)); otherwise the call
+                          returns DDT_ERR_INVALID_ARG                            */
   int32_t out_dtype;  /* ddt_dtype                                              */
   void* out;          /* [B, q_len, 64, 512]                                    */
   float* lse;         /* fp32 [B, q_len, 64] or NULL                            */

@@ -83,6 +83,13 @@ def test_host_argument_checks(lib):
     a.c_kv = fake
     a.ckv_row_stride = 500  # shorter than a row
     assert lib.ddt_verify_attn(ctypes.byref(a), None) == ddt.DDT_ERR_INVALID_ARG
+    a.ckv_row_stride = 512
+    # the softmax scale must be positive and finite (checked before any launch)
+    for bad in (0.0, -0.125, float("inf"), float("nan"), 3.0e38):
+        a.softmax_scale = bad
+        assert lib.ddt_verify_attn(ctypes.byref(a), None) == ddt.DDT_ERR_INVALID_ARG, bad
+        assert lib.ddt_verify_attn_noalloc(ctypes.byref(a), None) == ddt.DDT_ERR_INVALID_ARG, bad
+    a.softmax_scale = 0.0721
     a.B = 0
     assert lib.ddt_verify_attn(ctypes.byref(a), None) == ddt.DDT_OK
     # tree build: sizes, then null pointers; B = 0 is a no-op

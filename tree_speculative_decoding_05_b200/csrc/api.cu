@@ -290,7 +290,10 @@ static ddt_status check_attn_args(const ddt_attn_args* a) {
   if (!cache_strides_ok(a->B, a->capacity, a->ckv_batch_stride, a->ckv_row_stride,
                         a->kr_batch_stride, a->kr_row_stride))
     return DDT_ERR_INVALID_ARG;
-  if (!(a->softmax_scale == a->softmax_scale)) return DDT_ERR_INVALID_ARG;
+  // A positive, finite scale (and log2(e) times it): the kernel applies it after
+  // taking the maximum of the raw scores, which needs scale > 0.
+  const float scale_log2 = a->softmax_scale * 1.4426950408889634f;
+  if (!(a->softmax_scale > 0.0f) || !(scale_log2 <= 3.402823466e38f)) return DDT_ERR_INVALID_ARG;
   return DDT_OK;
 }
 

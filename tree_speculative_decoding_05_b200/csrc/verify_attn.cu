@@ -616,7 +616,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         // whose one tile may also reach prefix rows and rows below 0.
         const bool tree_pass = p.kv_mode == 2;
         const int lo = tree_pass ? INT_MIN : tile * kTK;
-        // Scaled, masked scores of 64-key chunk sc (log2 units).
+        // Masked raw scores of 64-key chunk sc (q . k; the scale, which the host
+        // checks is positive, is applied in the exponent's FMA and to the maximum).
         auto load_chunk = [&](int sc, float (&x)[64]) {
           uint32_t r0[32], r1[32];
           const uint32_t col = tmem + lane_addr + kTmemS + static_cast<uint32_t>(kSCols * sbuf + 64 * sc);
@@ -625,8 +626,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            x[c] = __uint_as_float(r0[c]) * p.scale_log2;
-            x[32 + c] = __uint_as_float(r1[c]) * p.scale_log2;
+            x[c] = __uint_as_float(r0[c]);
+            x[32 + c] = __uint_as_float(r1[c]);
           }
           const int key0 = kbase + 64 * sc;
           if (tree_pass || key0 + 64 > P || key0 < lo) {  // tree block, or the shifted last tile
@@ -661,7 +662,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
         named_barrier_sync(1, kSoftmaxThreads);
         // Every thread of this CTA has read S: release the buffer.
         if (kSChunks == 1 && t == 0) mbar_arrive_cluster(s_free_leader0 + 8u * sbuf);
-        mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]);
+        // log2 units from here: a positive scale commutes with the maximum
+        mx = fmaxf(mx, red_max[sb * 128 + (t ^ 64)]) * p.scale_log2;
         float factor = 1.f;
         bool rescale = false;
         if (m_ref == -INFINITY) {
@@ -681,8 +683,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(va::kThreads, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float e0 = fast_exp2(x[2 * c] - m_use);
-            const float e1 = fast_exp2(x[2 * c + 1] - m_use);
+            const float e0 = fast_exp2(fmaf(x[2 * c], p.scale_log2, -m_use));
+            const float e1 = fast_exp2(fmaf(x[2 * c + 1], p.scale_log2, -m_use));
             pk[c] = pack_bf16x2(e0, e1);
             l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
           }
