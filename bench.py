@@ -1158,11 +1158,22 @@ def main(argv=None) -> int:
     if rank == 0:
         peaks, peak_src = measured_peaks()
         timed_s = step_ms * args.steps / 1e3
-        use_sustained = timed_s > 2.0
+        clk = clocks.summary()
+        # The sustained peak (measured under the power cap) is the denominator when
+        # the timed region ran power-capped: over 2 s, or NVML samples inside it
+        # showing sw_power_cap with the median SM clock below 95 % of its maximum.
+        capped = (str(clk.get("source") or "").startswith("NVML")
+                  and "sw_power_cap" in clk.get("reasons", [])
+                  and clk.get("sm_mhz") and clk.get("sm_max_mhz")
+                  and clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
+        use_sustained = timed_s > 2.0 or bool(capped)
+        sustained_why = ("" if not use_sustained else
+                         " (timed region over 2 s)" if timed_s > 2.0 else
+                         f" (power-capped: median {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} "
+                         f"MHz with sw_power_cap in the timed region)")
         peak = peaks.get("bf16_tflops_sustained" if use_sustained else "bf16_tflops",
                          FALLBACK_BF16_TFLOPS)
         achieved = flops_local / (verify_ms_max * 1e-3) / 1e12
-        clk = clocks.summary()
         line = {
             "metric": METRIC,
             "value": flops_total / (step_ms_max * 1e-3) / 1e12,
@@ -1194,7 +1205,8 @@ def main(argv=None) -> int:
                              / (verify_ms_max * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_src} {'sustained' if use_sustained else 'burst'} bf16",
+                         "peak_source": f"{peak_src} {'sustained' if use_sustained else 'burst'} bf16"
+                                        f"{sustained_why}",
                          "traffic": measured_traffic(args.config),
                          "algorithmic_bytes": bytes_local,
                          "kernel": "verify_attn_kernel"},
