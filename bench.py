@@ -312,6 +312,25 @@ class ClockSampler:
                 "samples": len(sm), "source": "nvidia-smi every 100 ms around the timed region"}
 
 
+def choose_peak(peaks: dict, timed_s: float, clk: dict):
+    """The roofline's bf16 denominator: the sustained peak (measured under the
+    power cap) when the timed region ran power-capped, i.e. lasted over 2 s, or
+    its in-region NVML samples show sw_power_cap with the median SM clock below
+    95 % of its maximum; else the burst peak.  Returns (peak, sustained?, why)."""
+    capped = (str(clk.get("source") or "").startswith("NVML")
+              and "sw_power_cap" in (clk.get("reasons") or [])
+              and bool(clk.get("sm_mhz")) and bool(clk.get("sm_max_mhz"))
+              and clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
+    sustained = timed_s > 2.0 or capped
+    why = ("" if not sustained else
+           " (timed region over 2 s)" if timed_s > 2.0 else
+           f" (power-capped: median {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz with "
+           f"sw_power_cap in the timed region)")
+    peak = peaks.get("bf16_tflops_sustained" if sustained else "bf16_tflops",
+                     FALLBACK_BF16_TFLOPS)
+    return peak, sustained, why
+
+
 def physical_gpu_index(local: int) -> str:
     """nvidia-smi's index of the GPU this process uses."""
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -1159,20 +1178,7 @@ def main(argv=None) -> int:
         peaks, peak_src = measured_peaks()
         timed_s = step_ms * args.steps / 1e3
         clk = clocks.summary()
-        # The sustained peak (measured under the power cap) is the denominator when
-        # the timed region ran power-capped: over 2 s, or NVML samples inside it
-        # showing sw_power_cap with the median SM clock below 95 % of its maximum.
-        capped = (str(clk.get("source") or "").startswith("NVML")
-                  and "sw_power_cap" in clk.get("reasons", [])
-                  and clk.get("sm_mhz") and clk.get("sm_max_mhz")
-                  and clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
-        use_sustained = timed_s > 2.0 or bool(capped)
-        sustained_why = ("" if not use_sustained else
-                         " (timed region over 2 s)" if timed_s > 2.0 else
-                         f" (power-capped: median {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} "
-                         f"MHz with sw_power_cap in the timed region)")
-        peak = peaks.get("bf16_tflops_sustained" if use_sustained else "bf16_tflops",
-                         FALLBACK_BF16_TFLOPS)
+        peak, use_sustained, sustained_why = choose_peak(peaks, timed_s, clk)
         achieved = flops_local / (verify_ms_max * 1e-3) / 1e12
         line = {
             "metric": METRIC,

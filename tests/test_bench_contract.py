@@ -80,3 +80,24 @@ def test_clock_summary_takes_samples_inside_the_timed_region():
     s = c.summary()
     assert s["sm_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
     assert s["source"].startswith("nvidia-smi")
+
+
+def test_sustained_peak_only_for_a_power_capped_region():
+    """The burst peak is the roofline's denominator unless the timed region ran
+    power-capped: longer than 2 s, or NVML samples inside it with sw_power_cap
+    and the median SM clock below 95 % of its maximum."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    peaks = {"bf16_tflops": 1631.8, "bf16_tflops_sustained": 1400.0}
+    nvml = "NVML every ~2 ms inside the timed region"
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "source": nvml}
+    capped = {"sm_mhz": 1567.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "source": nvml}
+    assert bench.choose_peak(peaks, 0.05, full)[:2] == (1631.8, False)
+    assert bench.choose_peak(peaks, 0.3, capped)[:2] == (1400.0, True)
+    assert "power-capped" in bench.choose_peak(peaks, 0.3, capped)[2]
+    assert bench.choose_peak(peaks, 3.0, full)[:2] == (1400.0, True)
+    # the cap bit alone at full clock, or samples from outside the region, do not switch
+    assert bench.choose_peak(peaks, 0.3, dict(capped, sm_mhz=1940.0))[:2] == (1631.8, False)
+    smi = dict(capped, source="nvidia-smi every 100 ms around the timed region")
+    assert bench.choose_peak(peaks, 0.3, smi)[:2] == (1631.8, False)
