@@ -241,7 +241,8 @@ def verify_attn(q_lat: torch.Tensor, q_rope: torch.Tensor, c_kv: torch.Tensor,
                 stream=None, split_tail: bool = False):
     """Tree-verify MLA-absorb attention.  q_lat bf16 [B,Q,64,512], q_rope bf16
     [B,Q,64,64], c_kv bf16 [B,cap,512] and k_rope bf16 [B,cap,64] (rows may be
-    strided), prefix_lens int32 [B], mask from build_mask.  Returns (out, lse).
+    strided), prefix_lens int32 [B], mask from build_mask; softmax_scale must be
+    positive and finite (the library rejects anything else).  Returns (out, lse).
     split_tail=True computes it as a prefix pass, a tree-block pass and an LSE
     merge (ddt_verify_attn_split_tail) instead of one fused pass."""
     for t, n in ((q_lat, "q_lat"), (q_rope, "q_rope")):
